@@ -1,0 +1,22 @@
+"""fp64 CPU oracle for block-sparse causal attention (test infrastructure).
+
+This package is test infrastructure only.  It is a plain, slow, obviously
+correct restatement of what the block-sparse causal attention forward
+computes, written from the pages' statement of the method.  Only the test
+suite, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline and
+reference legs may import it; the CUDA product path never does, and the two
+share no code (the seeded input generator they both consume lives in its own
+module and contains none of the method's arithmetic).
+
+Modules:
+  layouts   -- kept-block sets for each pattern family, the SplitMix64
+               generator, CSR assembly, pair counts and reachability depth.
+  attention -- the masked-softmax definition (dense, tiny n), the same
+               definition restricted to its support (large n), and a pure
+               Python brute force for tiny inputs.
+
+Every function is pinned by a ``-m "not gpu"`` test against something other
+than itself (printed page values, closed forms, library routines, invariants,
+brute force); see ``tests/test_oracle_pins.py``.
+"""
+from . import layouts, attention  # noqa: F401
