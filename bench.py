@@ -1,0 +1,507 @@
+#!/usr/bin/env python3
+"""Benchmark of the block-sparse causal attention forward on B200.
+
+One step = one pass of the hot path over one batch of the headline workload:
+the layout is compiled once (it is data-independent, and its planning time is
+reported on its own, as the BF1 page times topology separately), then every
+step is one ``bsa_forward`` over all heads and query blocks.  ``value`` is the
+effective throughput 4*d*(kept token pairs) / time over the timed steps with
+inputs resident in HBM; ``e2e`` repeats the metric through the public API from
+pinned host buffers (layout compile + H2D of q, k, v + forward + D2H of o and
+lse inside every timed step).
+
+``python bench.py [--gpus N --steps K --warmup W] [--impl reference]``; under
+torchrun each rank runs an independent replica (the work items of this path
+share nothing, so there is no data-path collective) and rank 0 prints one JSON
+line with the max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_long_bsa_b200 import inputs as synth                  # noqa: E402
+from block_sparse_long_bsa_b200.workloads import WORKLOADS, ORDER, HEADLINE  # noqa: E402
+
+METRIC = "block-sparse attn fwd effective TFLOPS (4·d·kept pairs/s), % of B200 bf16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SRC = os.path.join(ROOT, "block_sparse_long_bsa_b200", "csrc", "bsa_fwd_sm100a.cu")
+THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                 0x100: "display_clock_setting"}
+
+
+# ------------------------------------------------------------------ helpers
+def kept_pairs_of_layout(row_ptr, col_idx, n, B, L):
+    """Token pairs allowed by a CSR layout (diagonal block counted causally)."""
+    nb = -(-n // B)
+    pairs = 0
+    for h in range(L):
+        for i in range(nb):
+            rows_i = min(n, (i + 1) * B) - i * B
+            for j in col_idx[row_ptr[h * nb + i]:row_ptr[h * nb + i + 1]]:
+                if j < i:
+                    pairs += rows_i * (min(n, (j + 1) * B) - j * B)
+                elif j == i:
+                    pairs += rows_i * (rows_i + 1) // 2
+    return pairs
+
+
+def workload_work(w, row_ptr, col_idx):
+    pairs_per_layout_head = []
+    nb = w.n_blocks
+    for h in range(w.layout_heads):
+        rp = row_ptr[h * nb:(h + 1) * nb + 1] - row_ptr[h * nb]
+        ci = col_idx[row_ptr[h * nb]:row_ptr[(h + 1) * nb]]
+        pairs_per_layout_head.append(kept_pairs_of_layout(rp, ci, w.n, w.B, 1))
+    reps = w.heads // w.layout_heads
+    pairs = sum(pairs_per_layout_head) * reps
+    flops = 4 * w.d * pairs
+    compulsory = 2 * (2 * w.heads * w.n * w.d + 2 * w.kv_heads * w.n * w.d) + 4 * w.heads * w.n
+    return pairs, flops, compulsory
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            pk = json.load(fh)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_sha():
+    with open(KERNEL_SRC, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, if it still
+    matches the kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"bsa_fwd_sm100a_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    sha = re.search(r"kernel_sha256:\s*([0-9a-f]{64})", text)
+    tr = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not sha or not tr or sha.group(1) != kernel_sha():
+        return None
+    return int(tr.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi samples (SM clock, max clock, throttle reasons) in a thread."""
+
+    def __init__(self, gpu_index: int, period_ms: int = 100):
+        self.cmd = ["nvidia-smi", "-i", str(gpu_index),
+                    "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                    "--format=csv,noheader,nounits", f"-lms", str(period_ms)]
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+            return
+        def reader():
+            for line in self.proc.stdout:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 4:
+                    try:
+                        self.samples.append((time.time(), float(parts[0]), float(parts[1]),
+                                             float(parts[2]) if parts[2] not in ("[N/A]", "N/A") else 0.0,
+                                             int(parts[3], 16) if parts[3].startswith("0x") else 0))
+                    except ValueError:
+                        pass
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        note = "timed region"
+        if len(win) < 3:
+            win = [s for s in self.samples if s[0] <= t1]
+            note = "warm-up and timed region"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": "none"}
+        loaded = [s for s in win if not (s[4] & 0x1)] or win
+        mhz = sorted(s[1] for s in loaded)
+        reasons = 0
+        for s in loaded:
+            reasons |= s[4]
+        names = [nm for bit, nm in THROTTLE_BITS.items() if reasons & bit]
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(s[2] for s in win),
+                "reasons": names, "power_w_max": max(s[3] for s in win),
+                "samples": len(loaded), "window": note}
+
+
+def threads_in_use():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        if info:
+            return max(int(i.get("num_threads", 1)) for i in info)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+def oracle_sample(w, sets, bits, budget_s, seed=7):
+    """Time the fp64 oracle on randomly drawn (head, query block) items until
+    about ``budget_s`` seconds of CPU work; returns (pairs, seconds, items)."""
+    from oracle import attention as OA
+    qf, kf, vf = (synth.bf16_bits_to_f64(x) for x in bits)   # upcast once, outside the clock
+    rng = np.random.default_rng(seed)
+    scale = 1.0 / math.sqrt(w.d)
+    pairs = 0
+    items = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < budget_s:
+        f = int(rng.integers(w.heads))
+        i = int(rng.integers(w.n_blocks))
+        row = sets[f % w.layout_heads][i]
+        OA.forward_block_rows(qf, kf, vf, sets, w.B, scale, f, i)
+        rows_i = min(w.n, (i + 1) * w.B) - i * w.B
+        for j in row:
+            if j < i:
+                pairs += rows_i * (min(w.n, (j + 1) * w.B) - j * w.B)
+            elif j == i:
+                pairs += rows_i * (rows_i + 1) // 2
+        items += 1
+    return pairs, time.perf_counter() - t0, items
+
+
+def sample_bits(w, heads_needed):
+    """Seeded inputs of the workload restricted to the first heads (CPU legs)."""
+    h = min(w.heads, heads_needed)
+    g = w.heads // w.kv_heads
+    kvh = max(1, -(-h // g))
+    q = synth.normal_bf16_bits((w.heads, w.n, w.d), synth.Q_SEED)[:h]
+    k = synth.normal_bf16_bits((w.kv_heads, w.n, w.d), synth.K_SEED)[:kvh]
+    v = synth.normal_bf16_bits((w.kv_heads, w.n, w.d), synth.V_SEED)[:kvh]
+    return q, k, v, h
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from oracle import layouts as OL
+    sets = OL.kept_sets_for(w)
+    q, k, v, h = sample_bits(w, 2)
+    import dataclasses
+    wh = dataclasses.replace(w, batch=1, q_heads=h, kv_heads_per_seq=max(1, h // (w.heads // w.kv_heads)))
+    per_step = max(0.5, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(wh, sets, (q, k, v), per_step / 4)
+    tot_pairs, tot_s, tot_items = 0, 0.0, 0
+    for s in range(args.steps):
+        p, t, it = oracle_sample(wh, sets, (q, k, v), per_step, seed=100 + s)
+        tot_pairs, tot_s, tot_items = tot_pairs + p, tot_s + t, tot_items + it
+    value = 4 * w.d * tot_pairs / tot_s / 1e12
+    cores = threads_in_use()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic N(0,1) bf16 inputs upcast exactly to fp64, seeds 0/1/2; layout seed 17",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{tot_items} random (head, query block) tiles of heads 0..{h - 1}, "
+                                   f"~{per_step:.1f} s of fp64 oracle work per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, gpus):
+    return {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads,
+            "kv_heads": w.kv_heads_per_seq, "n": w.n, "d": w.d, "B": w.B,
+            "layout_heads": w.layout_heads, "pattern": w.description,
+            "parallelism": "replicas" if gpus == 1 else f"replicas x{gpus} (independent batches per GPU)",
+            "l2": "inputs exceed the 126 MB L2 and a 256 MiB buffer is written between timed steps"}
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=HEADLINE, choices=ORDER)
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--only-device", action="store_true",
+                    help="device-timed leg only (no e2e, CPU baseline or other workloads); "
+                         "the form used for profiler captures")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import block_sparse_long_bsa_b200 as bsa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    bsa.load_library()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # --- layout (planning timed on its own)
+    t0 = time.perf_counter()
+    lay = bsa.Layout.for_workload(w, dev)
+    layout_ms = 1e3 * (time.perf_counter() - t0)
+    row_ptr, col_idx = lay.csr()
+    pairs, flops, compulsory = workload_work(w, row_ptr, col_idx)
+
+    # --- inputs (seeded, synthetic; resident in HBM for the device-timed value)
+    qb, kb, vb = synth.qkv_bits(w.heads, w.kv_heads, w.n, w.d)
+
+    def to_dev(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q, k, v = to_dev(qb), to_dev(kb), to_dev(vb)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.heads, w.n), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(w.d)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def fwd():
+        bsa.bsa_forward(q, k, v, lay.handle, w.B, w.n, w.heads, w.kv_heads, w.d, scale, o, lse, stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    time.sleep(0.3)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        fwd()
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    for s in range(args.steps):
+        flush.fill_(float(s))
+        starts[s].record(stream)
+        fwd()
+        ends[s].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall1 = time.time()
+    bsa.bsa_get_status(lay.handle)
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    local_total_ms = float(sum(step_ms))
+    total_ms = local_total_ms
+    if world > 1:
+        t = torch.tensor([local_total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    clocks = sampler.summary(wall0 - 0.05, wall1 + 0.05)
+
+    if args.only_device:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                              "config": workload_config(w, world), "partial": "device leg only"}),
+                  flush=True)
+        sampler.stop()
+        lay.close()
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # --- e2e through the public API from pinned host buffers
+    hq = torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hk = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    hv = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    ho = torch.empty(hq.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty((w.heads, w.n), dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    p = w.pattern
+
+    def e2e_step():
+        lay2 = bsa.Layout(p.kind, w.n, w.B, w.layout_heads, dev, window=p.window,
+                          global_first=p.global_first, dyadic_kmin=p.dyadic_kmin,
+                          density=p.density, seed=p.seed)
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        bsa.bsa_forward(dq, dk, dv, lay2.handle, w.B, w.n, w.heads, w.kv_heads, w.d, scale, o, lse, stream)
+        ho.copy_(o, non_blocking=True)
+        hl.copy_(lse, non_blocking=True)
+        return lay2
+
+    for _ in range(2):
+        e2e_step().close()
+    torch.cuda.synchronize()
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    keep = []
+    for _ in range(args.e2e_steps):
+        keep.append(e2e_step())
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    for l2 in keep:
+        l2.close()
+    e2e_ms = e_start.elapsed_time(e_end)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+    layout_bytes = 4 * (len(row_ptr) + len(col_idx) + len(row_ptr) - 1)
+    h2d = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + layout_bytes
+    d2h = o.numel() * 2 + lse.numel() * 4
+
+    # --- other workloads (same kernel, same protocol, fewer steps) on rank 0
+    per_config = {}
+    if rank == 0 and not args.no_per_config:
+        del hq, hk, hv, ho, hl, dq, dk, dv
+        for name in ORDER:
+            if name == w.name:
+                continue
+            per_config[name] = bench_other(WORKLOADS[name], dev, stream, flush, bsa, torch)
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    kernel_tflops = flops / (ms_per_step * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": kernel_tflops, "peak": peak, "unit": "TFLOP/s",
+                "frac": kernel_tflops / peak, "traffic": profiled_traffic(w.name),
+                "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                "algorithmic_flops_per_launch": flops,
+                "hbm_gbs_compulsory": compulsory / (ms_per_step * 1e-3) / 1e9}
+
+    # --- CPU oracle baseline (rank 0, one GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_budget > 0:
+        from oracle import layouts as OL
+        sets = OL.kept_sets_for(w)
+        sq, sk, sv, hh = sample_bits(w, 2)
+        import dataclasses
+        wh = dataclasses.replace(w, q_heads=hh, kv_heads_per_seq=max(1, hh // (w.heads // w.kv_heads)))
+        ps, secs, its = oracle_sample(wh, sets, (sq, sk, sv), args.cpu_budget)
+        cpu = {"value": 4 * w.d * ps / secs / 1e12, "unit": UNIT, "cores": threads_in_use(),
+               "kind": "oracle",
+               "sample": f"{its} random (head, query block) tiles of heads 0..{hh - 1} in {secs:.1f} s "
+                         f"(fp64 NumPy, BLAS threads as reported)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic N(0,1) bf16 from numpy default_rng seeds 0/1/2 (q/k/v); layout seed 17",
+            "config": workload_config(w, world),
+            "frac_of_peak": value / world / peak,
+            "layout_build_ms": layout_ms,
+            "kept_pairs": pairs,
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                    "includes": "layout compile+upload, H2D q/k/v, forward, D2H o/lse"},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "per_config": per_config,
+        }
+        print(json.dumps(line), flush=True)
+    sampler.stop()
+    lay.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_other(w, dev, stream, flush, bsa, torch, steps=10, warmup=3):
+    lay = bsa.Layout.for_workload(w, dev)
+    row_ptr, col_idx = lay.csr()
+    pairs, flops, compulsory = workload_work(w, row_ptr, col_idx)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    q = torch.randn((w.heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    k = torch.randn((w.kv_heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    v = torch.randn((w.kv_heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.heads, w.n), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(w.d)
+    ms = []
+    for s in range(warmup + steps):
+        flush.fill_(float(s))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        bsa.bsa_forward(q, k, v, lay.handle, w.B, w.n, w.heads, w.kv_heads, w.d, scale, o, lse, stream)
+        b.record(stream)
+        if s >= warmup:
+            ms.append((a, b))
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+    t = sorted(a.elapsed_time(b) for a, b in ms)
+    med = t[len(t) // 2]
+    lay.close()
+    del q, k, v, o, lse
+    return {"ms_median": med, "tflops": flops / (med * 1e-3) / 1e12, "kept_pairs": pairs,
+            "hbm_gbs_compulsory": compulsory / (med * 1e-3) / 1e9,
+            "data": "torch.randn on device, seed 1234"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

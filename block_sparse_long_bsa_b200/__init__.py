@@ -1,0 +1,232 @@
+"""Python binding of ``libbsa.so``: block-sparse causal attention forward on B200.
+
+Argument marshalling only.  Every step of the computation runs in the
+library's CUDA kernel or its host layout compiler; this module converts Python
+values and torch tensors to the C ABI declared in ``include/bsa.h`` and turns
+non-zero status codes into :class:`BsaError`.  There is no fallback: if the
+shared library is missing or cannot be loaded, every call raises.
+
+Names follow the C ABI: ``bsa_build_layout``, ``bsa_layout_csr``,
+``bsa_layout_order``, ``bsa_forward``, ``bsa_get_status``,
+``bsa_debug_timeout_probe``, ``bsa_free`` and ``bsa_last_error``; the
+``Layout`` class and ``attention`` are conveniences over them.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import numpy as np
+
+from .workloads import (PATTERN_BAND_GLOBAL, PATTERN_DYADIC, PATTERN_RANDOM,  # noqa: F401
+                        PATTERN_EXPLICIT)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+
+BSA_OK = 0
+STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "BSA_ERR_UNSUPPORTED",
+                4: "BSA_ERR_NONCAUSAL", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_OOM",
+                7: "BSA_ERR_DEVICE_TIMEOUT"}
+
+EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_order", "bsa_forward",
+            "bsa_get_status", "bsa_debug_timeout_probe", "bsa_free", "bsa_last_error"]
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+
+
+class bsa_pattern(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("global_first", ctypes.c_int32), ("dyadic_kmin", ctypes.c_int32),
+                ("density", ctypes.c_double), ("seed", ctypes.c_uint64),
+                ("mask", ctypes.POINTER(ctypes.c_uint8))]
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def load_library(path: str = LIB_PATH):
+    """Load (once) and return the ctypes handle; raises if the library is absent."""
+    global _lib
+    with _lib_lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(path):
+            raise RuntimeError(f"libbsa.so not found at {path}; build it with "
+                               "`python -m block_sparse_long_bsa_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I, U64, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint64, ctypes.c_float
+        lib.bsa_build_layout.argtypes = [ctypes.POINTER(bsa_pattern), I, I, I, I, ctypes.POINTER(P)]
+        lib.bsa_build_layout.restype = I
+        lib.bsa_layout_csr.argtypes = [P, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                       ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                       ctypes.POINTER(I), ctypes.POINTER(I)]
+        lib.bsa_layout_csr.restype = I
+        lib.bsa_layout_order.argtypes = [P, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                         ctypes.POINTER(I)]
+        lib.bsa_layout_order.restype = I
+        lib.bsa_forward.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P]
+        lib.bsa_forward.restype = I
+        lib.bsa_get_status.argtypes = [P, P]
+        lib.bsa_get_status.restype = I
+        lib.bsa_debug_timeout_probe.argtypes = [P, I, U64, P]
+        lib.bsa_debug_timeout_probe.restype = I
+        lib.bsa_free.argtypes = [P]
+        lib.bsa_free.restype = None
+        lib.bsa_last_error.argtypes = []
+        lib.bsa_last_error.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def bsa_last_error() -> str:
+    msg = load_library().bsa_last_error()
+    return msg.decode() if msg else ""
+
+
+def _check(status: int):
+    if status != BSA_OK:
+        raise BsaError(status, bsa_last_error())
+
+
+def _ptr(x) -> int:
+    """Device/host address of a torch tensor, or an int passed through."""
+    if x is None:
+        return 0
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> int:
+    if s is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except ImportError:
+            pass
+        return 0
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def bsa_build_layout(kind: int, n: int, B: int, layout_heads: int = 1, device: int = -1,
+                     window: int = 0, global_first: int = 0, dyadic_kmin: int = 2,
+                     density: float = 0.0, seed: int = 0, mask=None) -> int:
+    """Compile a pattern; returns the opaque layout handle (an int)."""
+    lib = load_library()
+    spec = bsa_pattern(kind, window, global_first, dyadic_kmin, density, seed & ((1 << 64) - 1), None)
+    keep = None
+    if mask is not None:
+        keep = np.ascontiguousarray(mask, dtype=np.uint8)
+        spec.mask = keep.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8))
+    out = ctypes.c_void_p()
+    _check(lib.bsa_build_layout(ctypes.byref(spec), n, B, layout_heads, device, ctypes.byref(out)))
+    return out.value
+
+
+def bsa_layout_csr(layout: int):
+    """Copies of (row_ptr, col_idx) as int32 numpy arrays."""
+    lib = load_library()
+    rp = ctypes.POINTER(ctypes.c_int32)()
+    ci = ctypes.POINTER(ctypes.c_int32)()
+    rows, nnz = ctypes.c_int(), ctypes.c_int()
+    _check(lib.bsa_layout_csr(layout, ctypes.byref(rp), ctypes.byref(ci), ctypes.byref(rows),
+                              ctypes.byref(nnz)))
+    row_ptr = np.ctypeslib.as_array(rp, shape=(rows.value + 1,)).copy()
+    col_idx = (np.ctypeslib.as_array(ci, shape=(nnz.value,)).copy() if nnz.value
+               else np.zeros(0, np.int32))
+    return row_ptr, col_idx
+
+
+def bsa_layout_order(layout: int) -> np.ndarray:
+    lib = load_library()
+    od = ctypes.POINTER(ctypes.c_int32)()
+    cnt = ctypes.c_int()
+    _check(lib.bsa_layout_order(layout, ctypes.byref(od), ctypes.byref(cnt)))
+    return np.ctypeslib.as_array(od, shape=(cnt.value,)).copy()
+
+
+def bsa_forward(q, k, v, layout: int, B: int, n: int, heads: int, kv_heads: int, d: int,
+                scale: float, o, lse, stream=None) -> None:
+    """Enqueue the forward on ``stream`` (default: torch's current stream)."""
+    lib = load_library()
+    _check(lib.bsa_forward(_ptr(q), _ptr(k), _ptr(v), layout, B, n, heads, kv_heads, d,
+                           ctypes.c_float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_get_status(layout: int, stream=None) -> None:
+    _check(load_library().bsa_get_status(layout, _stream(stream)))
+
+
+def bsa_debug_timeout_probe(layout: int, d: int, timeout_ns: int, stream=None) -> None:
+    _check(load_library().bsa_debug_timeout_probe(layout, d, timeout_ns, _stream(stream)))
+
+
+def bsa_free(layout: int) -> None:
+    if layout:
+        load_library().bsa_free(layout)
+
+
+class Layout:
+    """Owning wrapper of a layout handle (freed on ``close`` or collection)."""
+
+    def __init__(self, kind, n, B, layout_heads=1, device=-1, **pattern):
+        self.n, self.B, self.layout_heads, self.device = n, B, layout_heads, device
+        self.handle = bsa_build_layout(kind, n, B, layout_heads, device, **pattern)
+
+    @classmethod
+    def for_workload(cls, w, device=-1):
+        p = w.pattern
+        return cls(p.kind, w.n, w.B, w.layout_heads, device, window=p.window,
+                   global_first=p.global_first, dyadic_kmin=p.dyadic_kmin,
+                   density=p.density, seed=p.seed)
+
+    def csr(self):
+        return bsa_layout_csr(self.handle)
+
+    def order(self):
+        return bsa_layout_order(self.handle)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            bsa_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def attention(q, k, v, layout: Layout, scale: float | None = None, o=None, lse=None, stream=None):
+    """torch convenience: q [heads, n, d], k/v [kv_heads, n, d] bf16 CUDA tensors.
+
+    Allocates o / lse when not given and enqueues one ``bsa_forward``.
+    """
+    import torch
+    heads, n, d = q.shape
+    kv_heads = k.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((heads, n), dtype=torch.float32, device=q.device)
+    for t in (q, k, v, o):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise BsaError(1, "q, k, v, o must be contiguous bf16 tensors")
+    if lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise BsaError(1, "lse must be a contiguous float32 tensor")
+    bsa_forward(q, k, v, layout.handle, layout.B, n, heads, kv_heads, d, scale, o, lse, stream)
+    return o, lse

@@ -1,0 +1,730 @@
+// Block-sparse causal attention forward for B200 (sm_100a).
+//
+// What one CTA computes: one work item = (query tile, query block i).  A query
+// tile holds 128 query rows: one block of B = 128 tokens of one head, or, for
+// B = 64, the same block of two query heads that share a key/value head and a
+// layout row (grouped-query packing), else the block once plus a discarded
+// copy.  The CTA walks the CSR row of kept key blocks j ("Block Sparse
+// Attention in LLMs", section 6: for each query block, for each allowed key
+// block, a dense product; "Block-Sparse Attention", How It Works: dense work
+// inside an allowed block, skipped blocks never scored) and keeps a running
+// (FlashAttention-style, same page section 7) softmax so the n x n score
+// matrix never exists.
+//
+// Per kept block j:
+//   S = Q K_j^T                (tcgen05.mma, bf16 x bf16 -> fp32 in TMEM)
+//   diagonal block only: s[r][c] = -inf for key c > query r (the within-chunk
+//                        causal mask of "bsbr", Solution; BF1 section 3.1)
+//   m' = max(m, rowmax S); P = exp2((S - m') * scale*log2 e) as bf16 into TMEM
+//   O += P V_j                 (tcgen05.mma with A = P read from TMEM)
+// then o = O / l (bf16, TMA store) and lse = (m + log2 l) * ln 2.
+// The running max is only moved when a block's max exceeds it by more than
+// 2^8 (in exp2 units), which keeps P <= 256 (exact in bf16's range) and skips
+// almost every rescale of O; the final normalisation uses the same max as the
+// sum, so the result is the plain softmax.
+//
+// Roles (192 threads): warp 0 issues TMA loads (Q once, then K_j and V_j into a
+// ring of shared-memory slots); warp 1 owns TMEM and issues the MMAs from one
+// thread; warps 2-5 do the softmax, one query row per thread (a warp can only
+// reach its own quarter of the TMEM lanes: warp w serves rows 32*(w%4) ..).
+// Every wait on an mbarrier is bounded; when one runs out the kernel records
+// a status bit, every role stops issuing work, in-flight copies and MMAs are
+// drained, TMEM is released and the CTA returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace dev {
+
+constexpr int kThreads = 192;
+constexpr int kTileM = 128;          // query rows per CTA (one tcgen05 M=128 tile)
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.693147180559945309f;
+
+struct Params {
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  const int32_t* order;
+  float* lse;
+  uint32_t* status;
+  int n, nb, heads, L, group;
+  int pack;          // distinct heads per tile (1 or 2)
+  float scale_log2;  // scale * log2(e)
+  uint64_t timeout_ns;
+  int debug_never;
+};
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+struct Ctl {
+  volatile int* abort;   // shared: set once any wait of this CTA ran out
+  uint32_t* status;      // global status word
+  uint64_t timeout_ns;
+};
+
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort) return false;
+    if (globaltimer() - t0 > c.timeout_ns) {
+      *c.abort = 1;
+      atomicOr(c.status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+// Bounded wait for the completion of the phase with the given parity.
+__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const Ctl& c) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, c);
+}
+// Bounded wait that ignores the abort flag (used while draining on exit).
+__device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) return;
+  }
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// TMA (no multicast anywhere in this library).
+__device__ __forceinline__ void tma_prefetch(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_commit_and_wait() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// tcgen05 / TMEM
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+// D(tmem) (+)= A(smem desc) * B(smem desc)
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc)
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+// 16 consecutive 32-bit columns (each holding two bf16 values).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* u) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+// tcgen05 shared-memory matrix descriptor for a 128-byte-swizzled operand
+// (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B): start address,
+// leading and stride byte offsets (16-byte units), version 1, swizzle mode 2.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= uint64_t((addr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, A
+// K-major, B K-major (b_mn = 0) or MN-major (b_mn = 1), shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) |
+         (uint32_t(M >> 4) << 24);
+}
+
+// ---------------------------------------------------------------- the kernel
+template <int BLK, int HD, int NUM_S, int KVS>
+struct KernelShape {
+  static constexpr int kSubs = kTileM / BLK;                 // query blocks stacked in the tile
+  static constexpr int kAtoms = HD / 64;                     // 128-byte swizzle atoms along d
+  static constexpr int kQBytes = kTileM * HD * 2;
+  static constexpr int kTileBytes = BLK * HD * 2;            // one K or V block
+  static constexpr int kAtomRowsQ = kTileM * 128;            // bytes of one Q atom column
+  static constexpr int kAtomRowsKV = BLK * 128;              // bytes of one K/V atom column
+  static constexpr int kOffKV = kQBytes;
+  static constexpr int kOffBar = kOffKV + KVS * kTileBytes;
+  // barriers: q_full, kv_full[KVS], kv_empty[KVS], s_full[NUM_S], p_full[NUM_S], o_done, drain, never
+  static constexpr int kNumBars = 1 + 2 * KVS + 2 * NUM_S + 3;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemUsed = kOffMisc + 16;
+  static constexpr int kColS = 0;
+  static constexpr int kColO = NUM_S * BLK;
+  static constexpr int kColsNeeded = NUM_S * BLK + HD;
+  static constexpr uint32_t kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
+                                        : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
+  static constexpr uint32_t kIdescQK = idesc_bf16(kTileM, BLK, 0);
+  static constexpr uint32_t kIdescPV = idesc_bf16(kTileM, HD, 1);
+  static_assert(kColsNeeded <= 512, "TMEM budget");
+  static_assert(BLK == 64 || BLK == 128, "block size");
+  static_assert(HD == 64 || HD == 128, "head dim");
+};
+
+template <int BLK, int HD, int NUM_S, int KVS, int MIN_CTAS>
+__global__ void __launch_bounds__(kThreads, MIN_CTAS)
+    bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const Params p) {
+  using S = KernelShape<BLK, HD, NUM_S, KVS>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;               // 1024-byte aligned for SW128
+  uint8_t* gbase = smem_raw + (base - raw);
+
+  const uint32_t sQ = base;                                   // also the O staging buffer
+  const uint32_t sKV = base + S::kOffKV;
+  const uint32_t bar0 = base + S::kOffBar;
+  const uint32_t bQFull = bar0;
+  auto bKVFull = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bKVEmpty = [&](int s) { return bar0 + 8u * (1 + KVS + s); };
+  auto bSFull = [&](int s) { return bar0 + 8u * (1 + 2 * KVS + s); };
+  auto bPFull = [&](int s) { return bar0 + 8u * (1 + 2 * KVS + NUM_S + s); };
+  const uint32_t bODone = bar0 + 8u * (1 + 2 * KVS + 2 * NUM_S);
+  const uint32_t bDrain = bODone + 8u;
+  const uint32_t bNever = bODone + 16u;
+  volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(gbase + S::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + S::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const Ctl ctl{abort_flag, p.status, p.timeout_ns};
+
+  // ---- work item: (head group, rank in the longest-first order) -> query block
+  const int item = blockIdx.x;
+  const int hg = item / p.nb;
+  const int rank = item - hg * p.nb;
+  const int h0 = hg * p.pack;
+  const int lh = h0 % p.L;
+  const int kvh = h0 / p.group;
+  int row = 0, start = 0, len = 0;
+  bool diag_last = false;
+  if (!p.debug_never) {
+    row = __ldg(p.order + size_t(lh) * p.nb + rank);
+    const size_t r = size_t(lh) * p.nb + row;
+    start = __ldg(p.row_ptr + r);
+    len = __ldg(p.row_ptr + r + 1) - start;
+    diag_last = len > 0 && __ldg(p.col_idx + start + len - 1) == row;
+  }
+  auto head_of_sub = [&](int sub) { return h0 + (p.pack == 2 ? sub : 0); };
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    mbar_init(bQFull, 1);
+    for (int s = 0; s < KVS; ++s) {
+      mbar_init(bKVFull(s), 1);
+      mbar_init(bKVEmpty(s), 1);
+    }
+    for (int s = 0; s < NUM_S; ++s) {
+      mbar_init(bSFull(s), 1);
+      mbar_init(bPFull(s), 128);
+    }
+    mbar_init(bODone, 1);
+    mbar_init(bDrain, 1);
+    mbar_init(bNever, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    if (!p.debug_never) {
+      tma_prefetch(&tmQ);
+      tma_prefetch(&tmK);
+      tma_prefetch(&tmV);
+      tma_prefetch(&tmO);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(base + S::kOffMisc, S::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ================================================================ producer
+    if (lane == 0) {
+      int issued = 0;
+      bool q_issued = false;
+      bool ok = true;
+      if (p.debug_never) ok = wait(bNever, 0, ctl);
+      if (ok && len > 0) {
+        mbar_expect_tx(bQFull, S::kQBytes);
+        for (int sub = 0; sub < S::kSubs; ++sub)
+          for (int a = 0; a < S::kAtoms; ++a)
+            tma_load_3d(sQ + a * S::kAtomRowsQ + sub * BLK * 128, &tmQ, bQFull, a * 64, row * BLK,
+                        head_of_sub(sub));
+        q_issued = true;
+        for (int j = 0; j < len && ok; ++j) {
+          const int col = __ldg(p.col_idx + start + j);
+          for (int w = 0; w < 2; ++w) {
+            const int l = 2 * j + w;
+            const int slot = l % KVS;
+            if (l >= KVS) {
+              ok = wait(bKVEmpty(slot), ((l / KVS) - 1) & 1, ctl);
+              if (!ok) break;
+            }
+            mbar_expect_tx(bKVFull(slot), S::kTileBytes);
+            const CUtensorMap* m = w ? &tmV : &tmK;
+            for (int a = 0; a < S::kAtoms; ++a)
+              tma_load_3d(sKV + slot * S::kTileBytes + a * S::kAtomRowsKV, m, bKVFull(slot), a * 64,
+                          col * BLK, kvh);
+            ++issued;
+          }
+        }
+      }
+      // Never leave the CTA with copies in flight into its shared memory.
+      if (q_issued) wait_drain(bQFull, 0, 200000000ull);
+      for (int l = (issued > KVS ? issued - KVS : 0); l < issued; ++l)
+        wait_drain(bKVFull(l % KVS), (l / KVS) & 1, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      if (p.debug_never) ok = wait(bNever, 0, ctl);
+      if (ok && len > 0) {
+        ok = wait(bQFull, 0, ctl);
+        tc_fence_after();
+        auto issue_qk = [&](int j) -> bool {
+          const int l = 2 * j, slot = l % KVS;
+          if (!wait(bKVFull(slot), (l / KVS) & 1, ctl)) return false;
+          tc_fence_after();
+          const uint32_t d = tmem + S::kColS + (j % NUM_S) * BLK;
+          const uint32_t kb = sKV + slot * S::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t a = sw128_desc(sQ + (kk >> 2) * S::kAtomRowsQ + (kk & 3) * 32, 16, 1024);
+            const uint64_t b = sw128_desc(kb + (kk >> 2) * S::kAtomRowsKV + (kk & 3) * 32, 16, 1024);
+            mma_ss(d, a, b, S::kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bKVEmpty(slot));
+          tc_commit(bSFull(j % NUM_S));
+          return true;
+        };
+        auto issue_pv = [&](int j) -> bool {
+          if (!wait(bPFull(j % NUM_S), (j / NUM_S) & 1, ctl)) return false;
+          tc_fence_after();
+          const int l = 2 * j + 1, slot = l % KVS;
+          if (!wait(bKVFull(slot), (l / KVS) & 1, ctl)) return false;
+          tc_fence_after();
+          const uint32_t pa = tmem + S::kColS + (j % NUM_S) * BLK;
+          const uint32_t vb = sKV + slot * S::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < BLK / 16; ++kk) {
+            const uint64_t b = sw128_desc(vb + kk * 16 * 128, S::kAtomRowsKV, 1024);
+            mma_ts(tmem + S::kColO, pa + kk * 8, b, S::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bKVEmpty(slot));
+          tc_commit(bODone);
+          return true;
+        };
+        if (ok) {
+          if (NUM_S == 1) {
+            for (int j = 0; j < len && ok; ++j) ok = issue_qk(j) && issue_pv(j);
+          } else {
+            ok = issue_qk(0);
+            for (int j = 0; j < len && ok; ++j) {
+              if (j + 1 < len) ok = issue_qk(j + 1);
+              if (ok) ok = issue_pv(j);
+            }
+          }
+        }
+      }
+      // Wait for every MMA this thread issued before TMEM can be released.
+      tc_commit(bDrain);
+      wait_drain(bDrain, 0, 200000000ull);
+    }
+  } else {
+    // ================================================================ softmax
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;            // tile row = TMEM lane
+    const int sub = r / BLK;
+    const int rl = r - sub * BLK;            // row inside its query block
+    const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
+    const float sl2 = p.scale_log2;
+    float m2 = -INFINITY;                    // running max, in exp2 units
+    float l = 0.f;                           // running sum of P
+    bool ok = true;
+    if (p.debug_never) {
+      ok = wait(bNever, 0, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    for (int j = 0; ok && j < len; ++j) {
+      const int s = j % NUM_S;
+      ok = __all_sync(0xffffffffu, wait(bSFull(s), (j / NUM_S) & 1, ctl));
+      if (!ok) break;
+      tc_fence_after();
+      float sv[BLK];
+#pragma unroll
+      for (int c = 0; c < BLK / 32; ++c) tmem_ld32(lane_base + S::kColS + s * BLK + c * 32, sv + c * 32);
+      tmem_wait_ld();
+      if (diag_last && j == len - 1) {
+#pragma unroll
+        for (int c = 0; c < BLK; ++c)
+          if (c > rl) sv[c] = -INFINITY;
+      }
+      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+      for (int c = 4; c < BLK; c += 4) {
+        mx0 = fmaxf(mx0, sv[c]);
+        mx1 = fmaxf(mx1, sv[c + 1]);
+        mx2 = fmaxf(mx2, sv[c + 2]);
+        mx3 = fmaxf(mx3, sv[c + 3]);
+      }
+      const float mb = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      // Each row moves its own max (so rows never influence each other's
+      // rounding); the warp passes over O when any of its rows moved.
+      const bool need = j > 0 && mb > m2 + kRescaleThreshold;
+      const float m_new = (j == 0 || need) ? mb : m2;
+      const float alpha = need ? ex2(m2 - m_new) : 1.f;
+      const bool resc = __any_sync(0xffffffffu, need);
+      const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < BLK; c += 4) {
+        sv[c] = ex2(fmaf(sv[c], sl2, neg_m));
+        sv[c + 1] = ex2(fmaf(sv[c + 1], sl2, neg_m));
+        sv[c + 2] = ex2(fmaf(sv[c + 2], sl2, neg_m));
+        sv[c + 3] = ex2(fmaf(sv[c + 3], sl2, neg_m));
+        s0 += sv[c];
+        s1 += sv[c + 1];
+        s2 += sv[c + 2];
+        s3 += sv[c + 3];
+      }
+      l = l * alpha + ((s0 + s1) + (s2 + s3));
+      if (NUM_S == 2 && j > 0) {
+        // O must hold PV_{j-1} before it is rescaled (S_j may finish first).
+        ok = __all_sync(0xffffffffu, wait(bODone, (j - 1) & 1, ctl));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (resc) {
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          float ov[32];
+          tmem_ld32(lane_base + S::kColO + c * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+          tmem_st32(lane_base + S::kColO + c * 32, ov);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < BLK / 32; ++c) {
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
+        tmem_st16(lane_base + S::kColS + s * BLK + c * 16, u);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bPFull(s));
+      m2 = m_new;
+    }
+    if (ok && len > 0) {
+      ok = __all_sync(0xffffffffu, wait(bODone, (len - 1) & 1, ctl));
+      if (ok) tc_fence_after();
+    }
+    // ---- epilogue: o = O / l into the (now free) Q buffer, then TMA store
+    if (ok) {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        float ov[32];
+        if (len > 0) {
+          tmem_ld32(lane_base + S::kColO + c * 32, ov);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = 0.f;
+        }
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(ov[2 * e] * inv, ov[2 * e + 1] * inv);
+        const int atom = (c * 32) / 64;
+        const uint32_t rowaddr = sQ + atom * S::kAtomRowsQ + r * 128;
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const int chunk = ((c * 32) % 64) / 8 + qq;
+          st_shared_v4(rowaddr + ((chunk ^ (r & 7)) << 4), u[4 * qq], u[4 * qq + 1], u[4 * qq + 2],
+                       u[4 * qq + 3]);
+        }
+      }
+      const int t = row * BLK + rl;
+      if (sub < p.pack && t < p.n) {
+        const float lse = l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
+        p.lse[size_t(head_of_sub(sub)) * p.n + t] = lse;
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    named_sync(1, 128);
+    if (warp == 2 && lane == 0 && !*abort_flag && !p.debug_never) {
+      for (int sb = 0; sb < S::kSubs; ++sb) {
+        if (sb >= p.pack) break;
+        for (int a = 0; a < S::kAtoms; ++a)
+          tma_store_3d(&tmO, sQ + a * S::kAtomRowsQ + sb * BLK * 128, a * 64, row * BLK, head_of_sub(sb));
+      }
+      tma_store_commit_and_wait();
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, S::kTmemCols);
+  }
+}
+
+}  // namespace dev
+
+// ==================================================================== host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+int g_encode_status = BSA_OK;
+std::string g_encode_msg;
+
+int get_encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q{};
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+      g_encode_status = BSA_ERR_CUDA;
+      g_encode_msg = std::string("cuTensorMapEncodeTiled unavailable: ") + cudaGetErrorString(e);
+      return;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode_status != BSA_OK) return set_error(g_encode_status, g_encode_msg);
+  return BSA_OK;
+}
+
+// [slices][n][d] bf16, box of 64 columns x rows x 1 slice, 128-byte swizzle.
+int encode_map(CUtensorMap* m, const void* ptr, int slices, int n, int d, int rows) {
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(slices)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(n) * cuuint64_t(d) * 2};
+  cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
+  return BSA_OK;
+}
+
+template <int BLK, int HD, int NUM_S, int KVS, int MIN_CTAS>
+int launch_instance(const ForwardArgs& a, const dev::Params& p, int items) {
+  using S = dev::KernelShape<BLK, HD, NUM_S, KVS>;
+  auto kern = dev::bsa_fwd_kernel<BLK, HD, NUM_S, KVS, MIN_CTAS>;
+  // Ask for enough shared memory that no more than MIN_CTAS CTAs share an SM,
+  // so every resident CTA's TMEM allocation succeeds at once.
+  int smem = S::kSmemUsed + 1024;
+  const int floor_bytes = (228 * 1024) / (MIN_CTAS + 1) + 1024;
+  if (smem < floor_bytes) smem = floor_bytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+  CUtensorMap mq, mk, mv, mo;
+  std::memset(&mq, 0, sizeof(mq));
+  std::memset(&mk, 0, sizeof(mk));
+  std::memset(&mv, 0, sizeof(mv));
+  std::memset(&mo, 0, sizeof(mo));
+  if (!a.debug_never) {
+    int st = encode_map(&mq, a.q, a.heads, a.n, HD, BLK);
+    if (st == BSA_OK) st = encode_map(&mk, a.k, a.kv_heads, a.n, HD, BLK);
+    if (st == BSA_OK) st = encode_map(&mv, a.v, a.kv_heads, a.n, HD, BLK);
+    if (st == BSA_OK) st = encode_map(&mo, a.o, a.heads, a.n, HD, BLK);
+    if (st != BSA_OK) return st;
+  }
+  kern<<<items, dev::kThreads, smem, static_cast<cudaStream_t>(a.stream)>>>(mq, mk, mv, mo, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
+  return BSA_OK;
+}
+
+}  // namespace
+
+int launch_forward(const ForwardArgs& a) {
+  int st = get_encoder();
+  if (st != BSA_OK) return st;
+  const bsa_layout* L = a.layout;
+  dev::Params p{};
+  p.row_ptr = L->d_row_ptr;
+  p.col_idx = L->d_col_idx;
+  p.order = L->d_order;
+  p.lse = a.lse;
+  p.status = L->d_status;
+  p.n = a.n;
+  p.nb = L->nb;
+  p.heads = a.heads;
+  p.L = L->L;
+  p.group = a.heads / a.kv_heads;
+  p.pack = (a.B == 64 && p.group % 2 == 0 && L->L == 1) ? 2 : 1;
+  p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
+  p.timeout_ns = a.debug_never ? a.timeout_ns : 1000000000ull;   // 1 s: never reached in a correct run
+  p.debug_never = a.debug_never;
+  int items = (a.heads / p.pack) * L->nb;
+  if (items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
+  if (a.debug_never && items > 8) items = 8;
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 1, 2, 2>(a, p, items);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 1, 4, 2>(a, p, items);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2, 4, 2>(a, p, items);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2, 4, 2>(a, p, items);
+  return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
+}
+
+}  // namespace bsa

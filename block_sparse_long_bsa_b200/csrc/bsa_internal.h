@@ -1,0 +1,57 @@
+// Internal declarations shared by the host layout compiler, the C ABI and the
+// sm_100a kernel launcher.  Not part of the public interface.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "bsa.h"
+
+struct bsa_layout {
+  int n = 0;             // tokens per sequence
+  int B = 0;             // tokens per block
+  int nb = 0;            // blocks per sequence, ceil(n / B)
+  int L = 0;             // layout heads
+  int device = -1;       // device holding the uploaded arrays, -1 for host-only
+  int max_row = 0;       // longest row (kept blocks)
+  std::vector<int32_t> row_ptr;   // [L*nb + 1]
+  std::vector<int32_t> col_idx;   // [nnz]
+  std::vector<int32_t> order;     // [L*nb], longest row first per layout head
+  void* d_base = nullptr;         // single device allocation holding the arrays below
+  const int32_t* d_row_ptr = nullptr;
+  const int32_t* d_col_idx = nullptr;
+  const int32_t* d_order = nullptr;
+  uint32_t* d_status = nullptr;   // bit 0: a device wait ran out
+};
+
+namespace bsa {
+
+// Thread-local error message; returns the status for convenience.
+int set_error(int status, const std::string& msg);
+
+// Host layout compiler (bsa_layout.cpp).  Fills row_ptr/col_idx/order/max_row.
+int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out);
+
+// Device status bits.
+constexpr uint32_t kStatusTimeout = 1u;
+
+// Launch description handed to the kernel launcher (bsa_fwd_sm100a.cu).
+struct ForwardArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const bsa_layout* layout;
+  int B, n, heads, kv_heads, d;
+  float scale;
+  void* stream;
+  // diagnostics: every thread waits on a never-completed barrier
+  int debug_never;
+  uint64_t timeout_ns;
+};
+
+int launch_forward(const ForwardArgs& a);
+
+}  // namespace bsa

@@ -1,0 +1,161 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) block-sparse causal attention forward.
+ *
+ * What the library computes ("Block-Sparse Attention", ai-model-reference,
+ * sections "How It Works" and "Math Or Compute Schema"): the sequence of n
+ * tokens is cut into blocks of B tokens; query block i attends densely only
+ * to the key blocks its block mask M_B keeps; every dropped pair gets -inf
+ * before the softmax (scale 1/sqrt(d) in every shipped workload); inside the
+ * diagonal block the token-level causal mask applies (key u <= query t), as
+ * in "bsbr" ("Solution", the within-chunk causal mask M_in) and in BF1
+ * (section 3.1, the self block is read causally).  Block masks are compiled on
+ * the host into CSR form ("Block Sparse Attention in LLMs", section 6: the
+ * allowed_blocks list per query block).
+ *
+ * Conventions shared by every call:
+ *   - Every function returns a bsa_status (0 = BSA_OK); nothing throws or
+ *     aborts.  bsa_last_error() gives a message for the calling thread.
+ *   - Tensors are caller-owned device pointers: q is [heads][n][d] bf16,
+ *     k and v are [kv_heads][n][d] bf16, o is [heads][n][d] bf16 and lse is
+ *     [heads][n] float32, all contiguous.  A batch of b sequences with H
+ *     query heads and Hk key/value heads is passed folded: heads = b*H,
+ *     kv_heads = b*Hk.  Query slice f reads key/value slice
+ *     f / (heads / kv_heads) (contiguous grouped-query sharing) and layout
+ *     head f % layout_heads.
+ *   - Streams are caller-owned cudaStream_t values passed as void* (NULL is
+ *     the legacy default stream).  bsa_forward is asynchronous on that stream
+ *     and allocates nothing.
+ *   - A bsa_layout is library-owned: created only by bsa_build_layout (so it
+ *     is always valid and causal) and released only by bsa_free.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bsa_status {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, bad scale, wrong device ...  */
+  BSA_ERR_SHAPE = 2,          /* sizes inconsistent with each other or with the layout */
+  BSA_ERR_UNSUPPORTED = 3,    /* a size the kernels are not built for (B, d)           */
+  BSA_ERR_NONCAUSAL = 4,      /* an explicit block mask keeps a block j > i            */
+  BSA_ERR_CUDA = 5,           /* a CUDA runtime/driver call failed                     */
+  BSA_ERR_OOM = 6,            /* host or device allocation failed                      */
+  BSA_ERR_DEVICE_TIMEOUT = 7  /* a kernel wait ran out; the kernel returned early      */
+} bsa_status;
+
+/* Block-layout families.
+ *  BAND_GLOBAL: kept(i) = {max(0, i-window) .. i}, plus block 0 when
+ *      global_first != 0.  window = 0, global_first = 0 is BSBR's
+ *      within-chunk (block-diagonal) term ("bsbr", "Solution"); window >= 1
+ *      with block 0 is the local band plus global anchor block ("Block-Sparse
+ *      Attention", "How It Works"; "Block Sparse Attention in LLMs", 5B).
+ *  DYADIC: BAND_GLOBAL(window, global_first) plus i - 2^k for every
+ *      k >= dyadic_kmin with i - 2^k >= 0 (BF1, Method and section 3.1:
+ *      self, two local predecessors, the first block and dyadic predecessors;
+ *      window = 2, global_first = 1, dyadic_kmin = 2).  Sets, so overlaps
+ *      count once.
+ *  RANDOM: static random mask (BF1's "static-random graph" control, whose
+ *      generator is unpublished; this library's reading): the diagonal and
+ *      block 0 are always kept; row i keeps
+ *      min(i+1, max(mandatory, floor((ppm*(i+1) + 500000) / 1000000)))
+ *      blocks, ppm = round(density * 1e6); the others are drawn uniformly
+ *      without replacement from {1 .. i-1} by a partial Fisher-Yates shuffle
+ *      (draw t swaps candidate t with candidate t + x mod (i-1-t)), x being
+ *      successive SplitMix64 outputs from state seed + (h+1)*0x9E3779B97F4A7C15
+ *      for layout head h, rows taken in order.
+ *  EXPLICIT: the caller's block mask M_B ("Block-Sparse Attention", "Math Or
+ *      Compute Schema"): mask[h][i][j] != 0 keeps key block j for query
+ *      block i of layout head h.  Any kept j > i gives BSA_ERR_NONCAUSAL.
+ *      Rows may be empty (their output is o = 0, lse = -inf). */
+typedef enum bsa_pattern_kind {
+  BSA_PATTERN_BAND_GLOBAL = 0,
+  BSA_PATTERN_DYADIC = 1,
+  BSA_PATTERN_RANDOM = 2,
+  BSA_PATTERN_EXPLICIT = 3
+} bsa_pattern_kind;
+
+typedef struct bsa_pattern {
+  int32_t kind;          /* bsa_pattern_kind                                        */
+  int32_t window;        /* BAND_GLOBAL/DYADIC: local predecessors kept (>= 0)      */
+  int32_t global_first;  /* BAND_GLOBAL/DYADIC: nonzero keeps block 0               */
+  int32_t dyadic_kmin;   /* DYADIC: smallest exponent k of the offsets 2^k (>= 0)   */
+  double density;        /* RANDOM: target fraction of causal blocks, in [0, 1]     */
+  uint64_t seed;         /* RANDOM: generator seed                                  */
+  const uint8_t* mask;   /* EXPLICIT: host array [layout_heads][nb][nb], row-major,
+                            read only during bsa_build_layout; else ignored         */
+} bsa_pattern;
+
+typedef struct bsa_layout bsa_layout;   /* opaque */
+
+/* Compile a pattern into a block layout for sequences of n tokens in blocks of
+ * B tokens (nb = ceil(n / B); a shorter last block is allowed).
+ * layout_heads >= 1 separate layouts are built (the RANDOM family draws each
+ * from its own stream; the other families repeat the same rows).
+ * Produces, on the host: row_ptr[layout_heads*nb + 1] and col_idx[nnz]
+ * (rows in order head-major, columns strictly ascending, all <= the row's
+ * block index), and the longest-row-first order of each layout head's rows
+ * (ties broken by ascending row).  When device >= 0 the three arrays and a
+ * device status word are uploaded to that device synchronously; device = -1
+ * builds a host-only layout (inspection and tests; bsa_forward rejects it).
+ * On success *out owns everything; release it with bsa_free. */
+int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads,
+                     int device, bsa_layout** out);
+
+/* Read-only host view of a layout's CSR arrays; valid until bsa_free.
+ * rows = layout_heads * nb. */
+int bsa_layout_csr(const bsa_layout* layout, const int32_t** row_ptr,
+                   const int32_t** col_idx, int* rows, int* nnz);
+
+/* Read-only host view of the longest-row-first order: order[h*nb + r] is the
+ * query block processed at rank r for layout head h.  count = layout_heads*nb. */
+int bsa_layout_order(const bsa_layout* layout, const int32_t** order, int* count);
+
+/* Block-sparse causal attention forward on the caller's stream.
+ * For every folded query head f and token t (block i = t / B):
+ *   s_tu = scale * <q[f][t], k[g][u]>,  g = f / (heads / kv_heads),
+ *   over the keys u allowed by layout head f % layout_heads (block j of u kept
+ *   by block i, and j < i or u <= t);
+ *   lse[f][t] = ln sum_u exp(s_tu),  o[f][t] = sum_u exp(s_tu - lse) v[g][u].
+ * Rows with no allowed key get o = 0 and lse = -inf.
+ * Requirements (checked before anything is launched; violations return an
+ * error and launch nothing): layout built for this n and B on the current
+ * device; B in {64, 128}; d in {64, 128}; heads and kv_heads >= 1,
+ * heads % kv_heads == 0, heads % layout_heads == 0; scale finite and > 0;
+ * q, k, v, o non-null and 16-byte aligned; lse non-null and 4-byte aligned.
+ * o and lse must not overlap the inputs.  Launches one kernel; returns after
+ * enqueueing it.  A device-side wait that runs out (never expected) makes the
+ * kernel return early and is reported by bsa_get_status. */
+int bsa_forward(const void* q, const void* k, const void* v,
+                const bsa_layout* layout, int B, int n, int heads, int kv_heads,
+                int d, float scale, void* o, float* lse, void* stream);
+
+/* Synchronise `stream`, then read and clear the layout's device status word:
+ * BSA_OK, or BSA_ERR_DEVICE_TIMEOUT if any forward on this layout since the
+ * last call had a wait run out. */
+int bsa_get_status(const bsa_layout* layout, void* stream);
+
+/* Diagnostics: launch the forward kernel of this layout's shape in a mode
+ * where every thread waits on a barrier that nothing completes, with the
+ * given wait limit in nanoseconds (at most 10^9), so that the bounded-wait
+ * path runs: the kernel records BSA_ERR_DEVICE_TIMEOUT in the status word and
+ * returns; nothing is read or written besides the status word. */
+int bsa_debug_timeout_probe(const bsa_layout* layout, int d, uint64_t timeout_ns,
+                            void* stream);
+
+/* Release a layout and its device arrays (NULL is a no-op).  The caller must
+ * make sure no forward that uses it is still running. */
+void bsa_free(bsa_layout* layout);
+
+/* Message describing the last error returned on the calling thread. */
+const char* bsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H */

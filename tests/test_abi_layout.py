@@ -1,0 +1,145 @@
+"""Host-side checks of the C ABI (CPU only, no kernel launches).
+
+* the shared library loads and exports every function include/bsa.h declares;
+* the host layout compiler matches the oracle's independent builder bit for
+  bit (row_ptr, col_idx) on every workload pattern and on edge cases;
+* the longest-row-first order is a valid permutation in the stated order;
+* invalid specs return the documented status codes.
+"""
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import block_sparse_long_bsa_b200 as bsa
+from block_sparse_long_bsa_b200.workloads import WORKLOADS, ORDER
+from oracle import layouts as OL
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_long_bsa_b200 import build
+    build.build()
+    return bsa.load_library()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|void|const char\*)\s+(bsa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert "bsa_forward" in declared and "bsa_build_layout" in declared
+    out = subprocess.run(["nm", "-D", "--defined-only", bsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (bsa_\w+)", out))
+    missing = [f for f in declared if f not in exported]
+    assert not missing, missing
+    assert set(declared) == set(bsa.EXPORTED)
+
+
+def _csr_from_lib(kind, n, B, L, **kw):
+    lay = bsa.Layout(kind, n, B, L, -1, **kw)
+    rp, ci = lay.csr()
+    order = lay.order()
+    lay.close()
+    return rp, ci, order
+
+
+@pytest.mark.parametrize("name", ORDER)
+def test_layout_bit_exact_vs_oracle(lib, name):
+    w = WORKLOADS[name]
+    rp, ci, order = _csr_from_lib(w.pattern.kind, w.n, w.B, w.layout_heads,
+                                  window=w.pattern.window, global_first=w.pattern.global_first,
+                                  dyadic_kmin=w.pattern.dyadic_kmin, density=w.pattern.density,
+                                  seed=w.pattern.seed)
+    sets = OL.kept_sets_for(w)
+    orp, oci = OL.to_csr(sets)
+    np.testing.assert_array_equal(rp, np.array(orp, dtype=np.int32))
+    np.testing.assert_array_equal(ci, np.array(oci, dtype=np.int32))
+    _check_order(rp, order, w.layout_heads, w.n_blocks)
+
+
+def _check_order(rp, order, L, nb):
+    lens = np.diff(rp).reshape(L, nb)
+    order = order.reshape(L, nb)
+    for h in range(L):
+        assert sorted(order[h].tolist()) == list(range(nb))
+        ln = lens[h][order[h]]
+        assert np.all(ln[:-1] >= ln[1:])
+        # ties in length keep ascending block order
+        for a in range(nb - 1):
+            if ln[a] == ln[a + 1]:
+                assert order[h][a] < order[h][a + 1]
+
+
+@pytest.mark.parametrize("kind,n,B,L,kw", [
+    (OL.BAND_GLOBAL, 1, 64, 1, dict(window=3, global_first=1)),          # single token
+    (OL.BAND_GLOBAL, 1000, 64, 2, dict(window=0, global_first=0)),       # ragged, 16 blocks
+    (OL.BAND_GLOBAL, 777, 128, 1, dict(window=50, global_first=1)),      # window wider than n
+    (OL.DYADIC, 64 * 1000 + 5, 64, 1, dict(window=2, global_first=1, dyadic_kmin=2)),
+    (OL.DYADIC, 4096, 64, 3, dict(window=0, global_first=0, dyadic_kmin=0)),
+    (OL.RANDOM, 128 * 300, 128, 5, dict(density=0.25, seed=123456789)),
+    (OL.RANDOM, 64 * 50, 64, 2, dict(density=0.0, seed=1)),
+    (OL.RANDOM, 64 * 50 + 1, 64, 2, dict(density=1.0, seed=2 ** 64 - 1)),
+])
+def test_layout_edge_cases_bit_exact(lib, kind, n, B, L, kw):
+    rp, ci, order = _csr_from_lib(kind, n, B, L, **kw)
+    sets = OL.kept_sets(kind, n, B, L, **kw)
+    orp, oci = OL.to_csr(sets)
+    np.testing.assert_array_equal(rp, np.array(orp, dtype=np.int32))
+    np.testing.assert_array_equal(ci, np.array(oci, dtype=np.int32))
+    _check_order(rp, order, L, OL.n_blocks(n, B))
+
+
+def test_explicit_mask_bit_exact_and_noncausal(lib):
+    nb, B = 20, 64
+    rng = np.random.default_rng(0)
+    mask = (rng.random((2, nb, nb)) < 0.3) & np.tri(nb, dtype=bool)[None]
+    mask[1, 5, :] = False               # an empty row is allowed
+    rp, ci, order = _csr_from_lib(OL.EXPLICIT, nb * B, B, 2, mask=mask.astype(np.uint8))
+    sets = OL.kept_sets(OL.EXPLICIT, nb * B, B, 2, mask=mask.tolist())
+    orp, oci = OL.to_csr(sets)
+    np.testing.assert_array_equal(rp, orp)
+    np.testing.assert_array_equal(ci, oci)
+    bad = mask.copy()
+    bad[0, 3, 7] = True
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.Layout(OL.EXPLICIT, nb * B, B, 2, -1, mask=bad.astype(np.uint8))
+    assert ei.value.status == 4
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(kind=9, n=128, B=64), 1),
+    (dict(kind=0, n=0, B=64), 2),
+    (dict(kind=0, n=128, B=0), 2),
+    (dict(kind=0, n=128, B=64, layout_heads=0), 2),
+    (dict(kind=0, n=128, B=64, window=-1), 1),
+    (dict(kind=1, n=128, B=64, dyadic_kmin=-1), 1),
+    (dict(kind=2, n=128, B=64, density=1.5), 1),
+    (dict(kind=2, n=128, B=64, density=float("nan")), 1),
+    (dict(kind=3, n=128, B=64), 1),
+])
+def test_invalid_specs(lib, args, status):
+    kw = dict(args)
+    kind, n, B = kw.pop("kind"), kw.pop("n"), kw.pop("B")
+    L = kw.pop("layout_heads", 1)
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_build_layout(kind, n, B, L, -1, **kw)
+    assert ei.value.status == status
+    assert bsa.bsa_last_error()
+
+
+def test_forward_rejects_host_only_layout(lib):
+    lay = bsa.Layout(OL.BAND_GLOBAL, 256, 64, 1, -1, window=1, global_first=1)
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_forward(16, 16, 16, lay.handle, 64, 256, 1, 1, 64, 0.125, 16, 16, 0)
+    assert ei.value.status == 1
+    lay.close()
+    bsa.bsa_free(0)   # NULL is a no-op

