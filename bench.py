@@ -50,6 +50,8 @@ THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_p
 def kept_pairs_of_layout(row_ptr, col_idx, n, B, L):
     """Token pairs allowed by a CSR layout (diagonal block counted causally)."""
     nb = -(-n // B)
+    row_ptr = [int(x) for x in row_ptr]
+    col_idx = [int(x) for x in col_idx]
     pairs = 0
     for h in range(L):
         for i in range(nb):
@@ -408,6 +410,7 @@ def main():
         e2e_ms = float(t.item())
     e2e_value = world * flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
     layout_bytes = 4 * (len(row_ptr) + len(col_idx) + len(row_ptr) - 1)
+    pairs, flops = int(pairs), int(flops)
     h2d = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + layout_bytes
     d2h = o.numel() * 2 + lse.numel() * 4
 

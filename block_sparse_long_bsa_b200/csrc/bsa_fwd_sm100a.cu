@@ -50,14 +50,17 @@ constexpr int kThreads = 192;
 constexpr int kTileM = 128;          // query rows per CTA (one tcgen05 M=128 tile)
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.693147180559945309f;
+constexpr uint32_t kSuspendHintNs = 1000000;   // longest single suspension inside a wait
 
 struct Params {
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const int32_t* order;
+  __nv_bfloat16* o;
   float* lse;
   uint32_t* status;
   int n, nb, heads, L, group;
+  int items;         // work items in the longest-first list
   int pack;          // distinct heads per tile (1 or 2)
   float scale_log2;  // scale * log2(e)
   uint64_t timeout_ns;
@@ -89,37 +92,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
+}
+
+// Slow path of a bounded wait: poll (each try suspends the thread for up to
+// kSuspendHintNs or until the phase completes) until the phase completes, the
+// CTA's abort flag is raised, or `limit_ns` passes; on time-out record the
+// status bit and raise the abort flag.
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       uint32_t* status, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
 }
 
 struct Ctl {
   volatile int* abort;   // shared: set once any wait of this CTA ran out
   uint32_t* status;      // global status word
   uint64_t timeout_ns;
+  // Bounded wait for the completion of the phase with the given parity.
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, abort, status, timeout_ns);
+  }
 };
 
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, const Ctl& c) {
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*c.abort) return false;
-    if (globaltimer() - t0 > c.timeout_ns) {
-      *c.abort = 1;
-      atomicOr(c.status, kStatusTimeout);
-      return false;
-    }
-  }
-}
-// Bounded wait for the completion of the phase with the given parity.
-__device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity, const Ctl& c) {
-  if (mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, c);
-}
 // Bounded wait that ignores the abort flag (used while draining on exit).
 __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer();
@@ -295,8 +304,9 @@ struct KernelShape {
   static constexpr int kAtomRowsKV = BLK * 128;              // bytes of one K/V atom column
   static constexpr int kOffKV = kQBytes;
   static constexpr int kOffBar = kOffKV + KVS * kTileBytes;
-  // barriers: q_full, kv_full[KVS], kv_empty[KVS], s_full[NUM_S], p_full[NUM_S], o_done, drain, never
-  static constexpr int kNumBars = 1 + 2 * KVS + 2 * NUM_S + 3;
+  // barriers: q_full, q_free, kv_full[KVS], kv_empty[KVS], s_full[NUM_S],
+  //           p_full[NUM_S], o_done, o_free, drain, never
+  static constexpr int kNumBars = 2 + 2 * KVS + 2 * NUM_S + 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemUsed = kOffMisc + 16;
   static constexpr int kColS = 0;
@@ -311,56 +321,70 @@ struct KernelShape {
   static_assert(HD == 64 || HD == 128, "head dim");
 };
 
+// One work item = (head group, rank in its layout head's longest-first order).
+struct Item {
+  int row, start, len, h0, kvh;
+  bool diag_last;
+};
+
+__device__ __forceinline__ Item decode_item(const Params& p, int t) {
+  Item it;
+  const int hg = t / p.nb;
+  const int rank = t - hg * p.nb;
+  it.h0 = hg * p.pack;
+  it.kvh = it.h0 / p.group;
+  const int lh = it.h0 % p.L;
+  it.row = __ldg(p.order + size_t(lh) * p.nb + rank);
+  const size_t r = size_t(lh) * p.nb + it.row;
+  it.start = __ldg(p.row_ptr + r);
+  it.len = __ldg(p.row_ptr + r + 1) - it.start;
+  it.diag_last = it.len > 0 && __ldg(p.col_idx + it.start + it.len - 1) == it.row;
+  return it;
+}
+
+// Persistent schedule: CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... of the
+// longest-first list (alternating direction each round keeps the per-CTA
+// totals even when lengths fall along the list).
+__device__ __forceinline__ int item_at(int k) {
+  const int G = gridDim.x, c = blockIdx.x;
+  return k * G + ((k & 1) ? (G - 1 - c) : c);
+}
+
 template <int BLK, int HD, int NUM_S, int KVS, int MIN_CTAS>
 __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   const Params p) {
+                   const __grid_constant__ CUtensorMap tmV, const Params p) {
   using S = KernelShape<BLK, HD, NUM_S, KVS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;               // 1024-byte aligned for SW128
   uint8_t* gbase = smem_raw + (base - raw);
 
-  const uint32_t sQ = base;                                   // also the O staging buffer
+  const uint32_t sQ = base;
   const uint32_t sKV = base + S::kOffKV;
   const uint32_t bar0 = base + S::kOffBar;
   const uint32_t bQFull = bar0;
-  auto bKVFull = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto bKVEmpty = [&](int s) { return bar0 + 8u * (1 + KVS + s); };
-  auto bSFull = [&](int s) { return bar0 + 8u * (1 + 2 * KVS + s); };
-  auto bPFull = [&](int s) { return bar0 + 8u * (1 + 2 * KVS + NUM_S + s); };
-  const uint32_t bODone = bar0 + 8u * (1 + 2 * KVS + 2 * NUM_S);
-  const uint32_t bDrain = bODone + 8u;
-  const uint32_t bNever = bODone + 16u;
+  const uint32_t bQFree = bar0 + 8u;
+  auto bKVFull = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto bKVEmpty = [&](int s) { return bar0 + 8u * (2 + KVS + s); };
+  auto bSFull = [&](int s) { return bar0 + 8u * (2 + 2 * KVS + s); };
+  auto bPFull = [&](int s) { return bar0 + 8u * (2 + 2 * KVS + NUM_S + s); };
+  const uint32_t bODone = bar0 + 8u * (2 + 2 * KVS + 2 * NUM_S);
+  const uint32_t bOFree = bODone + 8u;
+  const uint32_t bDrain = bODone + 16u;
+  const uint32_t bNever = bODone + 24u;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(gbase + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + S::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const Ctl ctl{abort_flag, p.status, p.timeout_ns};
-
-  // ---- work item: (head group, rank in the longest-first order) -> query block
-  const int item = blockIdx.x;
-  const int hg = item / p.nb;
-  const int rank = item - hg * p.nb;
-  const int h0 = hg * p.pack;
-  const int lh = h0 % p.L;
-  const int kvh = h0 / p.group;
-  int row = 0, start = 0, len = 0;
-  bool diag_last = false;
-  if (!p.debug_never) {
-    row = __ldg(p.order + size_t(lh) * p.nb + rank);
-    const size_t r = size_t(lh) * p.nb + row;
-    start = __ldg(p.row_ptr + r);
-    len = __ldg(p.row_ptr + r + 1) - start;
-    diag_last = len > 0 && __ldg(p.col_idx + start + len - 1) == row;
-  }
-  auto head_of_sub = [&](int sub) { return h0 + (p.pack == 2 ? sub : 0); };
+  const int n_items = p.debug_never ? 0 : p.items;
 
   // ---- setup
   if (threadIdx.x == 0) {
     mbar_init(bQFull, 1);
+    mbar_init(bQFree, 1);
     for (int s = 0; s < KVS; ++s) {
       mbar_init(bKVFull(s), 1);
       mbar_init(bKVEmpty(s), 1);
@@ -370,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       mbar_init(bPFull(s), 128);
     }
     mbar_init(bODone, 1);
+    mbar_init(bOFree, 128);
     mbar_init(bDrain, 1);
     mbar_init(bNever, 1);
     *abort_flag = 0;
@@ -378,7 +403,6 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       tma_prefetch(&tmQ);
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
-      tma_prefetch(&tmO);
     }
   }
   if (warp == 1) {
@@ -393,37 +417,38 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
-      int issued = 0;
-      bool q_issued = false;
+      int issued = 0;        // K/V tile loads issued so far (ring position)
+      int q_loads = 0;       // Q tile loads issued so far
       bool ok = true;
-      if (p.debug_never) ok = wait(bNever, 0, ctl);
-      if (ok && len > 0) {
+      if (p.debug_never) ok = ctl.wait(bNever, 0);
+      for (int k = 0; ok; ++k) {
+        const int t = item_at(k);
+        if (t >= n_items) break;
+        const Item it = decode_item(p, t);
+        // the previous item's last QK^T has finished reading the Q buffer
+        if (k > 0 && !(ok = ctl.wait(bQFree, (k - 1) & 1))) break;
         mbar_expect_tx(bQFull, S::kQBytes);
         for (int sub = 0; sub < S::kSubs; ++sub)
           for (int a = 0; a < S::kAtoms; ++a)
-            tma_load_3d(sQ + a * S::kAtomRowsQ + sub * BLK * 128, &tmQ, bQFull, a * 64, row * BLK,
-                        head_of_sub(sub));
-        q_issued = true;
-        for (int j = 0; j < len && ok; ++j) {
-          const int col = __ldg(p.col_idx + start + j);
+            tma_load_3d(sQ + a * S::kAtomRowsQ + sub * BLK * 128, &tmQ, bQFull, a * 64,
+                        it.row * BLK, it.h0 + (p.pack == 2 ? sub : 0));
+        ++q_loads;
+        for (int j = 0; j < it.len && ok; ++j) {
+          const int col = __ldg(p.col_idx + it.start + j);
           for (int w = 0; w < 2; ++w) {
-            const int l = 2 * j + w;
-            const int slot = l % KVS;
-            if (l >= KVS) {
-              ok = wait(bKVEmpty(slot), ((l / KVS) - 1) & 1, ctl);
-              if (!ok) break;
-            }
+            const int l = issued, slot = l % KVS;
+            if (l >= KVS && !(ok = ctl.wait(bKVEmpty(slot), ((l / KVS) - 1) & 1))) break;
             mbar_expect_tx(bKVFull(slot), S::kTileBytes);
             const CUtensorMap* m = w ? &tmV : &tmK;
             for (int a = 0; a < S::kAtoms; ++a)
               tma_load_3d(sKV + slot * S::kTileBytes + a * S::kAtomRowsKV, m, bKVFull(slot), a * 64,
-                          col * BLK, kvh);
+                          col * BLK, it.kvh);
             ++issued;
           }
         }
       }
       // Never leave the CTA with copies in flight into its shared memory.
-      if (q_issued) wait_drain(bQFull, 0, 200000000ull);
+      if (q_loads > 0) wait_drain(bQFull, (q_loads - 1) & 1, 200000000ull);
       for (int l = (issued > KVS ? issued - KVS : 0); l < issued; ++l)
         wait_drain(bKVFull(l % KVS), (l / KVS) & 1, 200000000ull);
     }
@@ -431,15 +456,23 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     // ================================================================ MMA issuer
     if (lane == 0) {
       bool ok = true;
-      if (p.debug_never) ok = wait(bNever, 0, ctl);
-      if (ok && len > 0) {
-        ok = wait(bQFull, 0, ctl);
+      int kv = 0;            // K/V tiles consumed (ring position)
+      int s_cnt = 0;         // QK^T products issued (S buffer rotation)
+      int pv_cnt = 0;        // PV products issued
+      if (p.debug_never) ok = ctl.wait(bNever, 0);
+      for (int k = 0; ok; ++k) {
+        const int t = item_at(k);
+        if (t >= n_items) break;
+        const Item it = decode_item(p, t);
+        if (!(ok = ctl.wait(bQFull, k & 1))) break;
         tc_fence_after();
+        const int s_base = s_cnt;
         auto issue_qk = [&](int j) -> bool {
-          const int l = 2 * j, slot = l % KVS;
-          if (!wait(bKVFull(slot), (l / KVS) & 1, ctl)) return false;
+          const int l = kv + 2 * j, slot = l % KVS;
+          if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
           tc_fence_after();
-          const uint32_t d = tmem + S::kColS + (j % NUM_S) * BLK;
+          const int sb = (s_base + j) % NUM_S;
+          const uint32_t d = tmem + S::kColS + sb * BLK;
           const uint32_t kb = sKV + slot * S::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
@@ -448,16 +481,23 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             mma_ss(d, a, b, S::kIdescQK, kk > 0 ? 1u : 0u);
           }
           tc_commit(bKVEmpty(slot));
-          tc_commit(bSFull(j % NUM_S));
+          tc_commit(bSFull(sb));
+          if (j == it.len - 1) tc_commit(bQFree);      // last reader of this Q tile
           return true;
         };
         auto issue_pv = [&](int j) -> bool {
-          if (!wait(bPFull(j % NUM_S), (j / NUM_S) & 1, ctl)) return false;
+          const int sc = s_base + j, sb = sc % NUM_S;
+          if (!ctl.wait(bPFull(sb), (sc / NUM_S) & 1)) return false;
           tc_fence_after();
-          const int l = 2 * j + 1, slot = l % KVS;
-          if (!wait(bKVFull(slot), (l / KVS) & 1, ctl)) return false;
+          if (j == 0 && k > 0) {
+            // the previous item's epilogue has read O out of TMEM
+            if (!ctl.wait(bOFree, (k - 1) & 1)) return false;
+            tc_fence_after();
+          }
+          const int l = kv + 2 * j + 1, slot = l % KVS;
+          if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
           tc_fence_after();
-          const uint32_t pa = tmem + S::kColS + (j % NUM_S) * BLK;
+          const uint32_t pa = tmem + S::kColS + sb * BLK;
           const uint32_t vb = sKV + slot * S::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < BLK / 16; ++kk) {
@@ -468,17 +508,22 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           tc_commit(bODone);
           return true;
         };
-        if (ok) {
-          if (NUM_S == 1) {
-            for (int j = 0; j < len && ok; ++j) ok = issue_qk(j) && issue_pv(j);
-          } else {
-            ok = issue_qk(0);
-            for (int j = 0; j < len && ok; ++j) {
-              if (j + 1 < len) ok = issue_qk(j + 1);
-              if (ok) ok = issue_pv(j);
-            }
+        if (it.len == 0) {
+          // keep the O hand-over in step with the softmax warps
+          if (k > 0 && !(ok = ctl.wait(bOFree, (k - 1) & 1))) break;
+          tc_commit(bQFree);
+        } else if (NUM_S == 1) {
+          for (int j = 0; j < it.len && ok; ++j) ok = issue_qk(j) && issue_pv(j);
+        } else {
+          ok = issue_qk(0);
+          for (int j = 0; j < it.len && ok; ++j) {
+            if (j + 1 < it.len) ok = issue_qk(j + 1);
+            if (ok) ok = issue_pv(j);
           }
         }
+        kv += 2 * it.len;
+        s_cnt += it.len;
+        pv_cnt += it.len;
       }
       // Wait for every MMA this thread issued before TMEM can be released.
       tc_commit(bDrain);
@@ -492,130 +537,126 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     const int rl = r - sub * BLK;            // row inside its query block
     const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
     const float sl2 = p.scale_log2;
-    float m2 = -INFINITY;                    // running max, in exp2 units
-    float l = 0.f;                           // running sum of P
     bool ok = true;
-    if (p.debug_never) {
-      ok = wait(bNever, 0, ctl);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    for (int j = 0; ok && j < len; ++j) {
-      const int s = j % NUM_S;
-      ok = __all_sync(0xffffffffu, wait(bSFull(s), (j / NUM_S) & 1, ctl));
+    int s_cnt = 0, pv_cnt = 0;
+    if (p.debug_never) ok = __all_sync(0xffffffffu, ctl.wait(bNever, 0));
+    for (int k = 0; ok; ++k) {
+      const int t = item_at(k);
+      if (t >= n_items) break;
+      const Item it = decode_item(p, t);
+      float m2 = -INFINITY;                  // running max, in exp2 units
+      float l = 0.f;                         // running sum of P
+      for (int j = 0; ok && j < it.len; ++j) {
+        const int sc = s_cnt + j, s = sc % NUM_S;
+        ok = __all_sync(0xffffffffu, ctl.wait(bSFull(s), (sc / NUM_S) & 1));
+        if (!ok) break;
+        tc_fence_after();
+        float sv[BLK];
+#pragma unroll
+        for (int c = 0; c < BLK / 32; ++c) tmem_ld32(lane_base + S::kColS + s * BLK + c * 32, sv + c * 32);
+        tmem_wait_ld();
+        if (it.diag_last && j == it.len - 1) {
+#pragma unroll
+          for (int c = 0; c < BLK; ++c)
+            if (c > rl) sv[c] = -INFINITY;
+        }
+        float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+        for (int c = 4; c < BLK; c += 4) {
+          mx0 = fmaxf(mx0, sv[c]);
+          mx1 = fmaxf(mx1, sv[c + 1]);
+          mx2 = fmaxf(mx2, sv[c + 2]);
+          mx3 = fmaxf(mx3, sv[c + 3]);
+        }
+        const float mb = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        // Each row moves its own max (so rows never influence each other's
+        // rounding); the warp passes over O when any of its rows moved.
+        const bool need = j > 0 && mb > m2 + kRescaleThreshold;
+        const float m_new = (j == 0 || need) ? mb : m2;
+        const float alpha = need ? ex2(m2 - m_new) : 1.f;
+        const bool resc = __any_sync(0xffffffffu, need);
+        const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
+        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+        for (int c = 0; c < BLK; c += 4) {
+          sv[c] = ex2(fmaf(sv[c], sl2, neg_m));
+          sv[c + 1] = ex2(fmaf(sv[c + 1], sl2, neg_m));
+          sv[c + 2] = ex2(fmaf(sv[c + 2], sl2, neg_m));
+          sv[c + 3] = ex2(fmaf(sv[c + 3], sl2, neg_m));
+          s0 += sv[c];
+          s1 += sv[c + 1];
+          s2 += sv[c + 2];
+          s3 += sv[c + 3];
+        }
+        l = l * alpha + ((s0 + s1) + (s2 + s3));
+        if (NUM_S == 2 && j > 0) {
+          // O must hold PV_{j-1} before it is rescaled (S_j may finish first).
+          ok = __all_sync(0xffffffffu, ctl.wait(bODone, (pv_cnt + j - 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        if (resc) {
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c) {
+            float ov[32];
+            tmem_ld32(lane_base + S::kColO + c * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            tmem_st32(lane_base + S::kColO + c * 32, ov);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < BLK / 32; ++c) {
+          uint32_t u[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
+          tmem_st16(lane_base + S::kColS + s * BLK + c * 16, u);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bPFull(s));
+        m2 = m_new;
+      }
       if (!ok) break;
-      tc_fence_after();
-      float sv[BLK];
-#pragma unroll
-      for (int c = 0; c < BLK / 32; ++c) tmem_ld32(lane_base + S::kColS + s * BLK + c * 32, sv + c * 32);
-      tmem_wait_ld();
-      if (diag_last && j == len - 1) {
-#pragma unroll
-        for (int c = 0; c < BLK; ++c)
-          if (c > rl) sv[c] = -INFINITY;
-      }
-      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
-#pragma unroll
-      for (int c = 4; c < BLK; c += 4) {
-        mx0 = fmaxf(mx0, sv[c]);
-        mx1 = fmaxf(mx1, sv[c + 1]);
-        mx2 = fmaxf(mx2, sv[c + 2]);
-        mx3 = fmaxf(mx3, sv[c + 3]);
-      }
-      const float mb = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-      // Each row moves its own max (so rows never influence each other's
-      // rounding); the warp passes over O when any of its rows moved.
-      const bool need = j > 0 && mb > m2 + kRescaleThreshold;
-      const float m_new = (j == 0 || need) ? mb : m2;
-      const float alpha = need ? ex2(m2 - m_new) : 1.f;
-      const bool resc = __any_sync(0xffffffffu, need);
-      const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-      for (int c = 0; c < BLK; c += 4) {
-        sv[c] = ex2(fmaf(sv[c], sl2, neg_m));
-        sv[c + 1] = ex2(fmaf(sv[c + 1], sl2, neg_m));
-        sv[c + 2] = ex2(fmaf(sv[c + 2], sl2, neg_m));
-        sv[c + 3] = ex2(fmaf(sv[c + 3], sl2, neg_m));
-        s0 += sv[c];
-        s1 += sv[c + 1];
-        s2 += sv[c + 2];
-        s3 += sv[c + 3];
-      }
-      l = l * alpha + ((s0 + s1) + (s2 + s3));
-      if (NUM_S == 2 && j > 0) {
-        // O must hold PV_{j-1} before it is rescaled (S_j may finish first).
-        ok = __all_sync(0xffffffffu, wait(bODone, (j - 1) & 1, ctl));
+      if (it.len > 0) {
+        ok = __all_sync(0xffffffffu, ctl.wait(bODone, (pv_cnt + it.len - 1) & 1));
         if (!ok) break;
         tc_fence_after();
       }
-      if (resc) {
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          float ov[32];
-          tmem_ld32(lane_base + S::kColO + c * 32, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-          tmem_st32(lane_base + S::kColO + c * 32, ov);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < BLK / 32; ++c) {
-        uint32_t u[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
-        tmem_st16(lane_base + S::kColS + s * BLK + c * 16, u);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bPFull(s));
-      m2 = m_new;
-    }
-    if (ok && len > 0) {
-      ok = __all_sync(0xffffffffu, wait(bODone, (len - 1) & 1, ctl));
-      if (ok) tc_fence_after();
-    }
-    // ---- epilogue: o = O / l into the (now free) Q buffer, then TMA store
-    if (ok) {
+      // ---- epilogue: o = O / l straight from TMEM to global; lse alongside
+      const int tok = it.row * BLK + rl;
+      const bool store = sub < p.pack && tok < p.n;
+      const int head = it.h0 + (p.pack == 2 ? sub : 0);
+      uint4* orow = reinterpret_cast<uint4*>(p.o + (size_t(head) * p.n + (store ? tok : 0)) * HD);
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         float ov[32];
-        if (len > 0) {
+        if (it.len > 0) {
           tmem_ld32(lane_base + S::kColO + c * 32, ov);
           tmem_wait_ld();
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = 0.f;
         }
+        if (c == HD / 32 - 1) {
+          // O has been read: the next item's first PV may overwrite it
+          tc_fence_before();
+          mbar_arrive(bOFree);
+        }
         uint32_t u[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) u[e] = pack_bf16(ov[2 * e] * inv, ov[2 * e + 1] * inv);
-        const int atom = (c * 32) / 64;
-        const uint32_t rowaddr = sQ + atom * S::kAtomRowsQ + r * 128;
+        if (store) {
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int chunk = ((c * 32) % 64) / 8 + qq;
-          st_shared_v4(rowaddr + ((chunk ^ (r & 7)) << 4), u[4 * qq], u[4 * qq + 1], u[4 * qq + 2],
-                       u[4 * qq + 3]);
+          for (int qq = 0; qq < 4; ++qq)
+            orow[c * 4 + qq] = make_uint4(u[4 * qq], u[4 * qq + 1], u[4 * qq + 2], u[4 * qq + 3]);
         }
       }
-      const int t = row * BLK + rl;
-      if (sub < p.pack && t < p.n) {
-        const float lse = l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
-        p.lse[size_t(head_of_sub(sub)) * p.n + t] = lse;
-      }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    named_sync(1, 128);
-    if (warp == 2 && lane == 0 && !*abort_flag && !p.debug_never) {
-      for (int sb = 0; sb < S::kSubs; ++sb) {
-        if (sb >= p.pack) break;
-        for (int a = 0; a < S::kAtoms; ++a)
-          tma_store_3d(&tmO, sQ + a * S::kAtomRowsQ + sb * BLK * 128, a * 64, row * BLK, head_of_sub(sb));
-      }
-      tma_store_commit_and_wait();
+      if (store) p.lse[size_t(head) * p.n + tok] = l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
+      s_cnt += it.len;
+      pv_cnt += it.len;
     }
   }
 
@@ -668,7 +709,7 @@ int encode_map(CUtensorMap* m, const void* ptr, int slices, int n, int d, int ro
 }
 
 template <int BLK, int HD, int NUM_S, int KVS, int MIN_CTAS>
-int launch_instance(const ForwardArgs& a, const dev::Params& p, int items) {
+int launch_instance(const ForwardArgs& a, dev::Params p) {
   using S = dev::KernelShape<BLK, HD, NUM_S, KVS>;
   auto kern = dev::bsa_fwd_kernel<BLK, HD, NUM_S, KVS, MIN_CTAS>;
   // Ask for enough shared memory that no more than MIN_CTAS CTAs share an SM,
@@ -678,19 +719,25 @@ int launch_instance(const ForwardArgs& a, const dev::Params& p, int items) {
   if (smem < floor_bytes) smem = floor_bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-  CUtensorMap mq, mk, mv, mo;
+  int dev_id = 0, sms = 0;
+  e = cudaGetDevice(&dev_id);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
+  if (e != cudaSuccess || sms < 1) return set_error(BSA_ERR_CUDA, "cannot query the SM count");
+  CUtensorMap mq, mk, mv;
   std::memset(&mq, 0, sizeof(mq));
   std::memset(&mk, 0, sizeof(mk));
   std::memset(&mv, 0, sizeof(mv));
-  std::memset(&mo, 0, sizeof(mo));
+  int grid;
   if (!a.debug_never) {
     int st = encode_map(&mq, a.q, a.heads, a.n, HD, BLK);
     if (st == BSA_OK) st = encode_map(&mk, a.k, a.kv_heads, a.n, HD, BLK);
     if (st == BSA_OK) st = encode_map(&mv, a.v, a.kv_heads, a.n, HD, BLK);
-    if (st == BSA_OK) st = encode_map(&mo, a.o, a.heads, a.n, HD, BLK);
     if (st != BSA_OK) return st;
+    grid = p.items < sms * MIN_CTAS ? p.items : sms * MIN_CTAS;
+  } else {
+    grid = 8;
   }
-  kern<<<items, dev::kThreads, smem, static_cast<cudaStream_t>(a.stream)>>>(mq, mk, mv, mo, p);
+  kern<<<grid, dev::kThreads, smem, static_cast<cudaStream_t>(a.stream)>>>(mq, mk, mv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
   return BSA_OK;
@@ -717,13 +764,13 @@ int launch_forward(const ForwardArgs& a) {
   p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
   p.timeout_ns = a.debug_never ? a.timeout_ns : 1000000000ull;   // 1 s: never reached in a correct run
   p.debug_never = a.debug_never;
-  int items = (a.heads / p.pack) * L->nb;
-  if (items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
-  if (a.debug_never && items > 8) items = 8;
-  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 1, 2, 2>(a, p, items);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 1, 4, 2>(a, p, items);
-  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2, 4, 2>(a, p, items);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2, 4, 2>(a, p, items);
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.items = (a.heads / p.pack) * L->nb;
+  if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 1, 2, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 1, 4, 2>(a, p);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2, 4, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2, 4, 2>(a, p);
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 
