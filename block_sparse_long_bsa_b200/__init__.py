@@ -32,7 +32,8 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "B
                 7: "BSA_ERR_DEVICE_TIMEOUT"}
 
 EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_order", "bsa_forward",
-            "bsa_get_status", "bsa_debug_timeout_probe", "bsa_free", "bsa_last_error"]
+            "bsa_forward_noalloc", "bsa_get_status", "bsa_debug_timeout_probe", "bsa_free",
+            "bsa_last_error"]
 
 
 class BsaError(RuntimeError):
@@ -74,6 +75,8 @@ def load_library(path: str = LIB_PATH):
         lib.bsa_layout_order.restype = I
         lib.bsa_forward.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P]
         lib.bsa_forward.restype = I
+        lib.bsa_forward_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P]
+        lib.bsa_forward_noalloc.restype = I
         lib.bsa_get_status.argtypes = [P, P]
         lib.bsa_get_status.restype = I
         lib.bsa_debug_timeout_probe.argtypes = [P, I, U64, P]
@@ -162,6 +165,15 @@ def bsa_forward(q, k, v, layout: int, B: int, n: int, heads: int, kv_heads: int,
     lib = load_library()
     _check(lib.bsa_forward(_ptr(q), _ptr(k), _ptr(v), layout, B, n, heads, kv_heads, d,
                            ctypes.c_float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_forward_noalloc(q, k, v, layout: int, B: int, n: int, heads: int, kv_heads: int, d: int,
+                        scale: float, o, lse, stream=None) -> None:
+    """Allocation-free forward (see include/bsa.h): ``layout`` may be host-only;
+    its arrays are staged in the library's static device block."""
+    lib = load_library()
+    _check(lib.bsa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), layout, B, n, heads, kv_heads, d,
+                                   ctypes.c_float(scale), _ptr(o), _ptr(lse), _stream(stream)))
 
 
 def bsa_get_status(layout: int, stream=None) -> None:

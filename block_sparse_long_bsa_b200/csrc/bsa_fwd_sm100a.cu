@@ -774,4 +774,34 @@ int launch_forward(const ForwardArgs& a) {
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 
+int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int32_t* col_idx,
+                        const int32_t* order, uint32_t* status) {
+  int st = get_encoder();
+  if (st != BSA_OK) return st;
+  const bsa_layout* L = a.layout;
+  dev::Params p{};
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.order = order;
+  p.lse = a.lse;
+  p.status = status;
+  p.n = a.n;
+  p.nb = L->nb;
+  p.heads = a.heads;
+  p.L = L->L;
+  p.group = a.heads / a.kv_heads;
+  p.pack = (a.B == 64 && p.group % 2 == 0 && L->L == 1) ? 2 : 1;
+  p.scale_log2 = float(double(a.scale) * 1.4426950408889634);
+  p.timeout_ns = 1000000000ull;
+  p.debug_never = 0;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.items = (a.heads / p.pack) * L->nb;
+  if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 1, 2, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 1, 4, 2>(a, p);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2, 4, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2, 4, 2>(a, p);
+  return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
+}
+
 }  // namespace bsa

@@ -54,4 +54,9 @@ struct ForwardArgs {
 
 int launch_forward(const ForwardArgs& a);
 
+// Same launch with the layout arrays and status word at explicit device
+// addresses (the allocation-free entry point stages them itself).
+int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int32_t* col_idx,
+                        const int32_t* order, uint32_t* status);
+
 }  // namespace bsa

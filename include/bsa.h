@@ -147,6 +147,29 @@ int bsa_get_status(const bsa_layout* layout, void* stream);
 int bsa_debug_timeout_probe(const bsa_layout* layout, int d, uint64_t timeout_ns,
                             void* stream);
 
+/* Forward pass for callers that cannot allocate device memory.  This call has
+ * no counterpart on the pages that define the method; it exists for processes
+ * whose device memory belongs to someone else (a serving framework that
+ * reserved the GPU's memory in its own pool, a host application that lends the
+ * library only the buffers it passes in) and for code that must not allocate
+ * while running, since cudaMalloc/cudaFree can synchronise the whole device.
+ * Same arguments, checks and result as bsa_forward, except that `layout` may
+ * be host-only (built with device = -1) and nothing is allocated: on the
+ * caller's stream the call copies the layout's row_ptr, col_idx and order
+ * arrays into a block of device memory that the library declares statically
+ * (4 MiB of layout words plus a status word; every GPU that loads the library
+ * holds it until the process exits), clears the status word and launches the
+ * same kernel.  A layout needing more than 1,048,576 32-bit words
+ * (rows + 1 + nnz + rows) is rejected with BSA_ERR_SHAPE.  The first call on a
+ * device looks up that block's device address (cudaGetSymbolAddress), so make
+ * the first call on each device before any stream capture.  All calls share
+ * the block and each overwrites what the last one left: calls that overlap on
+ * the GPU race.  A device wait that runs out is recorded only in the shared
+ * block, not reported by this entry point. */
+int bsa_forward_noalloc(const void* q, const void* k, const void* v,
+                        const bsa_layout* layout, int B, int n, int heads, int kv_heads,
+                        int d, float scale, void* o, float* lse, void* stream);
+
 /* Release a layout and its device arrays (NULL is a no-op).  The caller must
  * make sure no forward that uses it is still running. */
 void bsa_free(bsa_layout* layout);
