@@ -294,29 +294,35 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 }
 
 // ---------------------------------------------------------------- the kernel
-template <int BLK, int HD, int NUM_S, int KVS>
+// Every kept key block is processed in chunks of 64 keys (one chunk for
+// B = 64, two for B = 128), so S is a 128 x 64 fp32 tile, two S buffers and the
+// O accumulator fit in 256 TMEM columns, and two CTAs share each SM.
+constexpr int kChunk = 64;
+
+template <int BLK, int HD, int KVS>
 struct KernelShape {
+  static constexpr int kCPB = BLK / kChunk;                  // chunks per kept block
   static constexpr int kSubs = kTileM / BLK;                 // query blocks stacked in the tile
   static constexpr int kAtoms = HD / 64;                     // 128-byte swizzle atoms along d
   static constexpr int kQBytes = kTileM * HD * 2;
-  static constexpr int kTileBytes = BLK * HD * 2;            // one K or V block
+  static constexpr int kTileBytes = kChunk * HD * 2;         // one 64-key chunk of K or V
   static constexpr int kAtomRowsQ = kTileM * 128;            // bytes of one Q atom column
-  static constexpr int kAtomRowsKV = BLK * 128;              // bytes of one K/V atom column
+  static constexpr int kAtomRowsKV = kChunk * 128;           // bytes of one K/V atom column
+  static constexpr int kWarpStage = 32 * 128;                // one warp's 32 rows x 64 columns of o
   static constexpr int kOffKV = kQBytes;
-  static constexpr int kOffBar = kOffKV + KVS * kTileBytes;
-  // barriers: q_full, q_free, kv_full[KVS], kv_empty[KVS], s_full[NUM_S],
-  //           p_full[NUM_S], o_done, o_free, drain, never
-  static constexpr int kNumBars = 2 + 2 * KVS + 2 * NUM_S + 4;
+  static constexpr int kOffStage = kOffKV + KVS * kTileBytes;
+  static constexpr int kOffBar = kOffStage + 4 * kWarpStage;
+  // barriers: q_full, q_free, kv_full[KVS], kv_empty[KVS], s_full[2], p_full[2],
+  //           o_done, o_free, drain, never
+  static constexpr int kNumBars = 2 + 2 * KVS + 4 + 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemUsed = kOffMisc + 16;
-  static constexpr int kColS = 0;
-  static constexpr int kColO = NUM_S * BLK;
-  static constexpr int kColsNeeded = NUM_S * BLK + HD;
-  static constexpr uint32_t kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
-                                        : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
-  static constexpr uint32_t kIdescQK = idesc_bf16(kTileM, BLK, 0);
+  static constexpr int kColS = 0;                            // S buffers: columns 0..63, 64..127
+  static constexpr int kColO = 2 * kChunk;
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr uint32_t kIdescQK = idesc_bf16(kTileM, kChunk, 0);
   static constexpr uint32_t kIdescPV = idesc_bf16(kTileM, HD, 1);
-  static_assert(kColsNeeded <= 512, "TMEM budget");
+  static_assert(2 * kChunk + HD <= 256, "TMEM budget");
   static_assert(BLK == 64 || BLK == 128, "block size");
   static_assert(HD == 64 || HD == 128, "head dim");
 };
@@ -350,26 +356,34 @@ __device__ __forceinline__ int item_at(int k) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-template <int BLK, int HD, int NUM_S, int KVS, int MIN_CTAS>
+template <int BLK, int HD, int KVS, int MIN_CTAS>
 __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const Params p) {
-  using S = KernelShape<BLK, HD, NUM_S, KVS>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = smem_addr(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;               // 1024-byte aligned for SW128
-  uint8_t* gbase = smem_raw + (base - raw);
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const Params p) {
+  using S = KernelShape<BLK, HD, KVS>;
+  constexpr int CPB = S::kCPB;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t base = smem_addr(smem_raw);
+  if (base & 1023u) {
+    // The 128-byte swizzle needs 1024-byte aligned tiles; refuse to run rather
+    // than compute garbage (never expected: dynamic shared memory starts aligned).
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
+    return;
+  }
+  uint8_t* gbase = smem_raw;
 
   const uint32_t sQ = base;
   const uint32_t sKV = base + S::kOffKV;
+  const uint32_t sStage = base + S::kOffStage;
   const uint32_t bar0 = base + S::kOffBar;
   const uint32_t bQFull = bar0;
   const uint32_t bQFree = bar0 + 8u;
   auto bKVFull = [&](int s) { return bar0 + 8u * (2 + s); };
   auto bKVEmpty = [&](int s) { return bar0 + 8u * (2 + KVS + s); };
   auto bSFull = [&](int s) { return bar0 + 8u * (2 + 2 * KVS + s); };
-  auto bPFull = [&](int s) { return bar0 + 8u * (2 + 2 * KVS + NUM_S + s); };
-  const uint32_t bODone = bar0 + 8u * (2 + 2 * KVS + 2 * NUM_S);
+  auto bPFull = [&](int s) { return bar0 + 8u * (2 + 2 * KVS + 2 + s); };
+  const uint32_t bODone = bar0 + 8u * (2 + 2 * KVS + 4);
   const uint32_t bOFree = bODone + 8u;
   const uint32_t bDrain = bODone + 16u;
   const uint32_t bNever = bODone + 24u;
@@ -389,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       mbar_init(bKVFull(s), 1);
       mbar_init(bKVEmpty(s), 1);
     }
-    for (int s = 0; s < NUM_S; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bSFull(s), 1);
       mbar_init(bPFull(s), 128);
     }
@@ -403,6 +417,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       tma_prefetch(&tmQ);
       tma_prefetch(&tmK);
       tma_prefetch(&tmV);
+      tma_prefetch(&tmO);
     }
   }
   if (warp == 1) {
@@ -417,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
-      int issued = 0;        // K/V tile loads issued so far (ring position)
+      int issued = 0;        // K/V chunk loads issued so far (ring position)
       int q_loads = 0;       // Q tile loads issued so far
       bool ok = true;
       if (p.debug_never) ok = ctl.wait(bNever, 0);
@@ -435,15 +450,17 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         ++q_loads;
         for (int j = 0; j < it.len && ok; ++j) {
           const int col = __ldg(p.col_idx + it.start + j);
-          for (int w = 0; w < 2; ++w) {
-            const int l = issued, slot = l % KVS;
-            if (l >= KVS && !(ok = ctl.wait(bKVEmpty(slot), ((l / KVS) - 1) & 1))) break;
-            mbar_expect_tx(bKVFull(slot), S::kTileBytes);
-            const CUtensorMap* m = w ? &tmV : &tmK;
-            for (int a = 0; a < S::kAtoms; ++a)
-              tma_load_3d(sKV + slot * S::kTileBytes + a * S::kAtomRowsKV, m, bKVFull(slot), a * 64,
-                          col * BLK, it.kvh);
-            ++issued;
+          for (int c = 0; c < CPB && ok; ++c) {
+            for (int w = 0; w < 2; ++w) {
+              const int l = issued, slot = l % KVS;
+              if (l >= KVS && !(ok = ctl.wait(bKVEmpty(slot), ((l / KVS) - 1) & 1))) break;
+              mbar_expect_tx(bKVFull(slot), S::kTileBytes);
+              const CUtensorMap* m = w ? &tmV : &tmK;
+              for (int a = 0; a < S::kAtoms; ++a)
+                tma_load_3d(sKV + slot * S::kTileBytes + a * S::kAtomRowsKV, m, bKVFull(slot), a * 64,
+                            col * BLK + c * kChunk, it.kvh);
+              ++issued;
+            }
           }
         }
       }
@@ -456,23 +473,22 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     // ================================================================ MMA issuer
     if (lane == 0) {
       bool ok = true;
-      int kv = 0;            // K/V tiles consumed (ring position)
+      int kv = 0;            // K/V chunks consumed (ring position)
       int s_cnt = 0;         // QK^T products issued (S buffer rotation)
-      int pv_cnt = 0;        // PV products issued
       if (p.debug_never) ok = ctl.wait(bNever, 0);
       for (int k = 0; ok; ++k) {
         const int t = item_at(k);
         if (t >= n_items) break;
         const Item it = decode_item(p, t);
+        const int nch = it.len * CPB;
         if (!(ok = ctl.wait(bQFull, k & 1))) break;
         tc_fence_after();
-        const int s_base = s_cnt;
-        auto issue_qk = [&](int j) -> bool {
-          const int l = kv + 2 * j, slot = l % KVS;
+        auto issue_qk = [&](int q) -> bool {
+          const int l = kv + 2 * q, slot = l % KVS;
           if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
           tc_fence_after();
-          const int sb = (s_base + j) % NUM_S;
-          const uint32_t d = tmem + S::kColS + sb * BLK;
+          const int sb = (s_cnt + q) & 1;
+          const uint32_t d = tmem + S::kColS + sb * kChunk;
           const uint32_t kb = sKV + slot * S::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
@@ -482,48 +498,45 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           }
           tc_commit(bKVEmpty(slot));
           tc_commit(bSFull(sb));
-          if (j == it.len - 1) tc_commit(bQFree);      // last reader of this Q tile
+          if (q == nch - 1) tc_commit(bQFree);      // last reader of this Q tile
           return true;
         };
-        auto issue_pv = [&](int j) -> bool {
-          const int sc = s_base + j, sb = sc % NUM_S;
-          if (!ctl.wait(bPFull(sb), (sc / NUM_S) & 1)) return false;
+        auto issue_pv = [&](int q) -> bool {
+          const int sc = s_cnt + q, sb = sc & 1;
+          if (!ctl.wait(bPFull(sb), (sc >> 1) & 1)) return false;
           tc_fence_after();
-          if (j == 0 && k > 0) {
+          if (q == 0 && k > 0) {
             // the previous item's epilogue has read O out of TMEM
             if (!ctl.wait(bOFree, (k - 1) & 1)) return false;
             tc_fence_after();
           }
-          const int l = kv + 2 * j + 1, slot = l % KVS;
+          const int l = kv + 2 * q + 1, slot = l % KVS;
           if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
           tc_fence_after();
-          const uint32_t pa = tmem + S::kColS + sb * BLK;
+          const uint32_t pa = tmem + S::kColS + sb * kChunk;
           const uint32_t vb = sKV + slot * S::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < BLK / 16; ++kk) {
+          for (int kk = 0; kk < kChunk / 16; ++kk) {
             const uint64_t b = sw128_desc(vb + kk * 16 * 128, S::kAtomRowsKV, 1024);
-            mma_ts(tmem + S::kColO, pa + kk * 8, b, S::kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + S::kColO, pa + kk * 8, b, S::kIdescPV, (q > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(bKVEmpty(slot));
           tc_commit(bODone);
           return true;
         };
-        if (it.len == 0) {
+        if (nch == 0) {
           // keep the O hand-over in step with the softmax warps
           if (k > 0 && !(ok = ctl.wait(bOFree, (k - 1) & 1))) break;
           tc_commit(bQFree);
-        } else if (NUM_S == 1) {
-          for (int j = 0; j < it.len && ok; ++j) ok = issue_qk(j) && issue_pv(j);
         } else {
           ok = issue_qk(0);
-          for (int j = 0; j < it.len && ok; ++j) {
-            if (j + 1 < it.len) ok = issue_qk(j + 1);
-            if (ok) ok = issue_pv(j);
+          for (int q = 0; q < nch && ok; ++q) {
+            if (q + 1 < nch) ok = issue_qk(q + 1);
+            if (ok) ok = issue_pv(q);
           }
         }
-        kv += 2 * it.len;
-        s_cnt += it.len;
-        pv_cnt += it.len;
+        kv += 2 * nch;
+        s_cnt += nch;
       }
       // Wait for every MMA this thread issued before TMEM can be released.
       tc_commit(bDrain);
@@ -536,33 +549,39 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     const int sub = r / BLK;
     const int rl = r - sub * BLK;            // row inside its query block
     const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
+    const uint32_t stage = sStage + q4 * S::kWarpStage;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    int s_cnt = 0, pv_cnt = 0;
+    int s_cnt = 0;                           // chunks seen (S buffer rotation, o_done phase)
+    bool stores_pending = false;
     if (p.debug_never) ok = __all_sync(0xffffffffu, ctl.wait(bNever, 0));
     for (int k = 0; ok; ++k) {
       const int t = item_at(k);
       if (t >= n_items) break;
       const Item it = decode_item(p, t);
+      const int nch = it.len * CPB;
+      const int diag_first = it.diag_last ? nch - CPB : nch;   // first chunk of the diagonal block
       float m2 = -INFINITY;                  // running max, in exp2 units
       float l = 0.f;                         // running sum of P
-      for (int j = 0; ok && j < it.len; ++j) {
-        const int sc = s_cnt + j, s = sc % NUM_S;
-        ok = __all_sync(0xffffffffu, ctl.wait(bSFull(s), (sc / NUM_S) & 1));
+      for (int q = 0; ok && q < nch; ++q) {
+        const int sc = s_cnt + q, s = sc & 1;
+        ok = __all_sync(0xffffffffu, ctl.wait(bSFull(s), (sc >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
-        float sv[BLK];
-#pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) tmem_ld32(lane_base + S::kColS + s * BLK + c * 32, sv + c * 32);
+        float sv[kChunk];
+        tmem_ld32(lane_base + S::kColS + s * kChunk, sv);
+        tmem_ld32(lane_base + S::kColS + s * kChunk + 32, sv + 32);
         tmem_wait_ld();
-        if (it.diag_last && j == it.len - 1) {
+        if (q >= diag_first) {
+          // causal mask inside the diagonal block: key (chunk offset + c) > row
+          const int lim = rl - (q - diag_first) * kChunk;
 #pragma unroll
-          for (int c = 0; c < BLK; ++c)
-            if (c > rl) sv[c] = -INFINITY;
+          for (int c = 0; c < kChunk; ++c)
+            if (c > lim) sv[c] = -INFINITY;
         }
         float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
 #pragma unroll
-        for (int c = 4; c < BLK; c += 4) {
+        for (int c = 4; c < kChunk; c += 4) {
           mx0 = fmaxf(mx0, sv[c]);
           mx1 = fmaxf(mx1, sv[c + 1]);
           mx2 = fmaxf(mx2, sv[c + 2]);
@@ -571,14 +590,14 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         const float mb = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
         // Each row moves its own max (so rows never influence each other's
         // rounding); the warp passes over O when any of its rows moved.
-        const bool need = j > 0 && mb > m2 + kRescaleThreshold;
-        const float m_new = (j == 0 || need) ? mb : m2;
+        const bool need = q > 0 && mb > m2 + kRescaleThreshold;
+        const float m_new = (q == 0 || need) ? mb : m2;
         const float alpha = need ? ex2(m2 - m_new) : 1.f;
         const bool resc = __any_sync(0xffffffffu, need);
         const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
         float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-        for (int c = 0; c < BLK; c += 4) {
+        for (int c = 0; c < kChunk; c += 4) {
           sv[c] = ex2(fmaf(sv[c], sl2, neg_m));
           sv[c + 1] = ex2(fmaf(sv[c + 1], sl2, neg_m));
           sv[c + 2] = ex2(fmaf(sv[c + 2], sl2, neg_m));
@@ -589,9 +608,9 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           s3 += sv[c + 3];
         }
         l = l * alpha + ((s0 + s1) + (s2 + s3));
-        if (NUM_S == 2 && j > 0) {
-          // O must hold PV_{j-1} before it is rescaled (S_j may finish first).
-          ok = __all_sync(0xffffffffu, ctl.wait(bODone, (pv_cnt + j - 1) & 1));
+        if (q > 0) {
+          // O must hold PV_{q-1} before it is rescaled (S_q may finish first).
+          ok = __all_sync(0xffffffffu, ctl.wait(bODone, (sc - 1) & 1));
           if (!ok) break;
           tc_fence_after();
         }
@@ -607,11 +626,11 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           }
         }
 #pragma unroll
-        for (int c = 0; c < BLK / 32; ++c) {
+        for (int c = 0; c < kChunk / 32; ++c) {
           uint32_t u[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) u[e] = pack_bf16(sv[c * 32 + 2 * e], sv[c * 32 + 2 * e + 1]);
-          tmem_st16(lane_base + S::kColS + s * BLK + c * 16, u);
+          tmem_st16(lane_base + S::kColS + s * kChunk + c * 16, u);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -619,45 +638,64 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         m2 = m_new;
       }
       if (!ok) break;
-      if (it.len > 0) {
-        ok = __all_sync(0xffffffffu, ctl.wait(bODone, (pv_cnt + it.len - 1) & 1));
+      if (nch > 0) {
+        ok = __all_sync(0xffffffffu, ctl.wait(bODone, (s_cnt + nch - 1) & 1));
         if (!ok) break;
         tc_fence_after();
       }
-      // ---- epilogue: o = O / l straight from TMEM to global; lse alongside
-      const int tok = it.row * BLK + rl;
-      const bool store = sub < p.pack && tok < p.n;
-      const int head = it.h0 + (p.pack == 2 ? sub : 0);
-      uint4* orow = reinterpret_cast<uint4*>(p.o + (size_t(head) * p.n + (store ? tok : 0)) * HD);
+      // ---- epilogue: o = O / l, 64 columns at a time through this warp's
+      // 32-row staging box and a TMA store; lse straight to global
+      const int r0 = q4 * 32;                // first row of this warp
+      const int sub0 = r0 / BLK;
+      const int tok0 = it.row * BLK + (r0 - sub0 * BLK);
+      const int head0 = it.h0 + (p.pack == 2 ? sub0 : 0);
+      const bool warp_stores = sub0 < p.pack;
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        float ov[32];
-        if (it.len > 0) {
-          tmem_ld32(lane_base + S::kColO + c * 32, ov);
+      for (int a = 0; a < S::kAtoms; ++a) {
+        float ov[64];
+        if (nch > 0) {
+          tmem_ld32(lane_base + S::kColO + a * 64, ov);
+          tmem_ld32(lane_base + S::kColO + a * 64 + 32, ov + 32);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = 0.f;
+          for (int e = 0; e < 64; ++e) ov[e] = 0.f;
         }
-        if (c == HD / 32 - 1) {
+        if (a == S::kAtoms - 1) {
           // O has been read: the next item's first PV may overwrite it
           tc_fence_before();
           mbar_arrive(bOFree);
         }
-        uint32_t u[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(ov[2 * e] * inv, ov[2 * e + 1] * inv);
-        if (store) {
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq)
-            orow[c * 4 + qq] = make_uint4(u[4 * qq], u[4 * qq + 1], u[4 * qq + 2], u[4 * qq + 3]);
+        if (stores_pending) {
+          // the previous store out of this staging box must have read it
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+          stores_pending = false;
         }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          st_shared_v4(stage + lane * 128 + ((ch ^ (lane & 7)) << 4),
+                       pack_bf16(ov[8 * ch] * inv, ov[8 * ch + 1] * inv),
+                       pack_bf16(ov[8 * ch + 2] * inv, ov[8 * ch + 3] * inv),
+                       pack_bf16(ov[8 * ch + 4] * inv, ov[8 * ch + 5] * inv),
+                       pack_bf16(ov[8 * ch + 6] * inv, ov[8 * ch + 7] * inv));
+        fence_proxy_async();
+        __syncwarp();
+        if (warp_stores && lane == 0 && !*abort_flag) {
+          tma_store_3d(&tmO, stage, a * 64, tok0, head0);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        stores_pending = true;
       }
-      if (store) p.lse[size_t(head) * p.n + tok] = l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
-      s_cnt += it.len;
-      pv_cnt += it.len;
+      const int tok = it.row * BLK + rl;
+      if (sub < p.pack && tok < p.n)
+        p.lse[size_t(it.h0 + (p.pack == 2 ? sub : 0)) * p.n + tok] =
+            l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
+      s_cnt += nch;
     }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
 
   // ---- teardown
@@ -708,13 +746,13 @@ int encode_map(CUtensorMap* m, const void* ptr, int slices, int n, int d, int ro
   return BSA_OK;
 }
 
-template <int BLK, int HD, int NUM_S, int KVS, int MIN_CTAS>
+template <int BLK, int HD, int KVS, int MIN_CTAS>
 int launch_instance(const ForwardArgs& a, dev::Params p) {
-  using S = dev::KernelShape<BLK, HD, NUM_S, KVS>;
-  auto kern = dev::bsa_fwd_kernel<BLK, HD, NUM_S, KVS, MIN_CTAS>;
+  using S = dev::KernelShape<BLK, HD, KVS>;
+  auto kern = dev::bsa_fwd_kernel<BLK, HD, KVS, MIN_CTAS>;
   // Ask for enough shared memory that no more than MIN_CTAS CTAs share an SM,
   // so every resident CTA's TMEM allocation succeeds at once.
-  int smem = S::kSmemUsed + 1024;
+  int smem = S::kSmemUsed;
   const int floor_bytes = (228 * 1024) / (MIN_CTAS + 1) + 1024;
   if (smem < floor_bytes) smem = floor_bytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -723,21 +761,23 @@ int launch_instance(const ForwardArgs& a, dev::Params p) {
   e = cudaGetDevice(&dev_id);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
   if (e != cudaSuccess || sms < 1) return set_error(BSA_ERR_CUDA, "cannot query the SM count");
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   std::memset(&mq, 0, sizeof(mq));
   std::memset(&mk, 0, sizeof(mk));
   std::memset(&mv, 0, sizeof(mv));
+  std::memset(&mo, 0, sizeof(mo));
   int grid;
   if (!a.debug_never) {
     int st = encode_map(&mq, a.q, a.heads, a.n, HD, BLK);
-    if (st == BSA_OK) st = encode_map(&mk, a.k, a.kv_heads, a.n, HD, BLK);
-    if (st == BSA_OK) st = encode_map(&mv, a.v, a.kv_heads, a.n, HD, BLK);
+    if (st == BSA_OK) st = encode_map(&mk, a.k, a.kv_heads, a.n, HD, dev::kChunk);
+    if (st == BSA_OK) st = encode_map(&mv, a.v, a.kv_heads, a.n, HD, dev::kChunk);
+    if (st == BSA_OK) st = encode_map(&mo, a.o, a.heads, a.n, HD, 32);
     if (st != BSA_OK) return st;
     grid = p.items < sms * MIN_CTAS ? p.items : sms * MIN_CTAS;
   } else {
     grid = 8;
   }
-  kern<<<grid, dev::kThreads, smem, static_cast<cudaStream_t>(a.stream)>>>(mq, mk, mv, p);
+  kern<<<grid, dev::kThreads, smem, static_cast<cudaStream_t>(a.stream)>>>(mq, mk, mv, mo, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
   return BSA_OK;
@@ -767,10 +807,10 @@ int launch_forward(const ForwardArgs& a) {
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
-  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 1, 2, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 1, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2, 4, 2>(a, p);
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 4, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 8, 2>(a, p);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 4, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 8, 2>(a, p);
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 
@@ -797,10 +837,10 @@ int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int3
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
-  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 1, 2, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 1, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2, 4, 2>(a, p);
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 4, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 8, 2>(a, p);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 4, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 8, 2>(a, p);
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 
