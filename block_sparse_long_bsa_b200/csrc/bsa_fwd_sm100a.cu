@@ -312,11 +312,12 @@ struct KernelShape {
   static constexpr int kOffKV = kQBytes;
   static constexpr int kOffStage = kOffKV + KVS * kTileBytes;
   static constexpr int kOffBar = kOffStage + 4 * kWarpStage;
-  // barriers: q_full, q_free, kv_full[KVS], kv_empty[KVS], s_full[2], p_full[2],
-  //           o_done, o_free, drain, never
-  static constexpr int kNumBars = 2 + 2 * KVS + 4 + 4;
+  // barriers: q_full, q_free, kv_full[KVS], s_full[2], p_full[2],
+  //           o_done[2] (PV products with even / odd index), o_free, drain, never
+  static constexpr int kNumBars = 2 + KVS + 4 + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemUsed = kOffMisc + 16;
+  static constexpr int kOffHist = kOffMisc + 16;             // producer's ring history [KVS] int
+  static constexpr int kSmemUsed = kOffHist + 4 * KVS;
   static constexpr int kColS = 0;                            // S buffers: columns 0..63, 64..127
   static constexpr int kColO = 2 * kChunk;
   static constexpr uint32_t kTmemCols = 256;
@@ -325,6 +326,7 @@ struct KernelShape {
   static_assert(2 * kChunk + HD <= 256, "TMEM budget");
   static_assert(BLK == 64 || BLK == 128, "block size");
   static_assert(HD == 64 || HD == 128, "head dim");
+  static_assert(KVS == 4, "the ring-slot hand-off relies on exactly four slots");
 };
 
 // One work item = (head group, rank in its layout head's longest-first order).
@@ -380,15 +382,20 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   const uint32_t bQFull = bar0;
   const uint32_t bQFree = bar0 + 8u;
   auto bKVFull = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto bKVEmpty = [&](int s) { return bar0 + 8u * (2 + KVS + s); };
-  auto bSFull = [&](int s) { return bar0 + 8u * (2 + 2 * KVS + s); };
-  auto bPFull = [&](int s) { return bar0 + 8u * (2 + 2 * KVS + 2 + s); };
-  const uint32_t bODone = bar0 + 8u * (2 + 2 * KVS + 4);
-  const uint32_t bOFree = bODone + 8u;
-  const uint32_t bDrain = bODone + 16u;
-  const uint32_t bNever = bODone + 24u;
+  auto bSFull = [&](int s) { return bar0 + 8u * (2 + KVS + s); };
+  auto bPFull = [&](int s) { return bar0 + 8u * (2 + KVS + 2 + s); };
+  // PV product j completes barrier o_done[j & 1]: each barrier then advances
+  // once per two products, so a softmax warp that skips waiting on some of
+  // them is never two phases behind when it does wait (S_q is committed after
+  // PV_{q-2}, and PV_{q+1} cannot finish before P_{q+1} exists).
+  const uint32_t bODone0 = bar0 + 8u * (2 + KVS + 4);
+  auto bODone = [&](int j) { return bODone0 + 8u * (j & 1); };
+  const uint32_t bOFree = bODone0 + 16u;
+  const uint32_t bDrain = bODone0 + 24u;
+  const uint32_t bNever = bODone0 + 32u;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(gbase + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + S::kOffMisc + 4);
+  int* ring_hist = reinterpret_cast<int*>(gbase + S::kOffHist);   // chunk index | (is V) << 31
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -399,15 +406,13 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   if (threadIdx.x == 0) {
     mbar_init(bQFull, 1);
     mbar_init(bQFree, 1);
-    for (int s = 0; s < KVS; ++s) {
-      mbar_init(bKVFull(s), 1);
-      mbar_init(bKVEmpty(s), 1);
-    }
+    for (int s = 0; s < KVS; ++s) mbar_init(bKVFull(s), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bSFull(s), 1);
       mbar_init(bPFull(s), 128);
     }
-    mbar_init(bODone, 1);
+    mbar_init(bODone(0), 1);
+    mbar_init(bODone(1), 1);
     mbar_init(bOFree, 128);
     mbar_init(bDrain, 1);
     mbar_init(bNever, 1);
@@ -434,6 +439,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     if (lane == 0) {
       int issued = 0;        // K/V chunk loads issued so far (ring position)
       int q_loads = 0;       // Q tile loads issued so far
+      int chunks = 0;        // chunks of earlier items (global chunk index base)
       bool ok = true;
       if (p.debug_never) ok = ctl.wait(bNever, 0);
       for (int k = 0; ok; ++k) {
@@ -448,21 +454,35 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             tma_load_3d(sQ + a * S::kAtomRowsQ + sub * BLK * 128, &tmQ, bQFull, a * 64,
                         it.row * BLK, it.h0 + (p.pack == 2 ? sub : 0));
         ++q_loads;
-        for (int j = 0; j < it.len && ok; ++j) {
-          const int col = __ldg(p.col_idx + it.start + j);
-          for (int c = 0; c < CPB && ok; ++c) {
-            for (int w = 0; w < 2; ++w) {
-              const int l = issued, slot = l % KVS;
-              if (l >= KVS && !(ok = ctl.wait(bKVEmpty(slot), ((l / KVS) - 1) & 1))) break;
-              mbar_expect_tx(bKVFull(slot), S::kTileBytes);
-              const CUtensorMap* m = w ? &tmV : &tmK;
-              for (int a = 0; a < S::kAtoms; ++a)
-                tma_load_3d(sKV + slot * S::kTileBytes + a * S::kAtomRowsKV, m, bKVFull(slot), a * 64,
-                            col * BLK + c * kChunk, it.kvh);
-              ++issued;
-            }
+        // Chunk q of the item owns ring positions 2q (K) and 2q + 1 (V) after
+        // the item's base, so every chunk occupies exactly two positions.
+        const int nch = it.len * CPB;
+        for (int idx = 0; idx < 2 * nch && ok; ++idx) {
+          const int q = idx >> 1;
+          const bool is_v = idx & 1;
+          const int key0 = __ldg(p.col_idx + it.start + q / CPB) * BLK + (q % CPB) * kChunk;
+          const int l = issued, slot = l % KVS;
+          if (l >= KVS) {
+            // The slot frees when the product that read its previous tile is
+            // done: QK^T of that chunk for a K tile (s_full), PV for a V tile
+            // (o_done).  A slot holds chunk c, then chunk c + 2 of the same
+            // kind, so with four slots the next completion of the same
+            // barrier needs the very tile loaded here and the phase test can
+            // be neither behind nor ahead by two phases.
+            const int prev = ring_hist[slot];
+            const int pc = prev & 0x7fffffff;
+            const uint32_t bar = (prev < 0) ? bODone(pc) : bSFull(pc & 1);
+            if (!(ok = ctl.wait(bar, (pc >> 1) & 1))) break;
           }
+          ring_hist[slot] = (is_v ? int(0x80000000u) : 0) | (chunks + q);
+          mbar_expect_tx(bKVFull(slot), S::kTileBytes);
+          const CUtensorMap* m = is_v ? &tmV : &tmK;
+          for (int a = 0; a < S::kAtoms; ++a)
+            tma_load_3d(sKV + slot * S::kTileBytes + a * S::kAtomRowsKV, m, bKVFull(slot), a * 64, key0,
+                        it.kvh);
+          ++issued;
         }
+        chunks += nch;
       }
       // Never leave the CTA with copies in flight into its shared memory.
       if (q_loads > 0) wait_drain(bQFull, (q_loads - 1) & 1, 200000000ull);
@@ -483,8 +503,11 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         const int nch = it.len * CPB;
         if (!(ok = ctl.wait(bQFull, k & 1))) break;
         tc_fence_after();
+        // ring positions of K_q and V_q
+        auto k_pos = [&](int q) { return kv + 2 * q; };
+        auto v_pos = [&](int q) { return kv + 2 * q + 1; };
         auto issue_qk = [&](int q) -> bool {
-          const int l = kv + 2 * q, slot = l % KVS;
+          const int l = k_pos(q), slot = l % KVS;
           if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
           tc_fence_after();
           const int sb = (s_cnt + q) & 1;
@@ -496,7 +519,6 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             const uint64_t b = sw128_desc(kb + (kk >> 2) * S::kAtomRowsKV + (kk & 3) * 32, 16, 1024);
             mma_ss(d, a, b, S::kIdescQK, kk > 0 ? 1u : 0u);
           }
-          tc_commit(bKVEmpty(slot));
           tc_commit(bSFull(sb));
           if (q == nch - 1) tc_commit(bQFree);      // last reader of this Q tile
           return true;
@@ -510,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             if (!ctl.wait(bOFree, (k - 1) & 1)) return false;
             tc_fence_after();
           }
-          const int l = kv + 2 * q + 1, slot = l % KVS;
+          const int l = v_pos(q), slot = l % KVS;
           if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
           tc_fence_after();
           const uint32_t pa = tmem + S::kColS + sb * kChunk;
@@ -520,8 +542,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             const uint64_t b = sw128_desc(vb + kk * 16 * 128, S::kAtomRowsKV, 1024);
             mma_ts(tmem + S::kColO, pa + kk * 8, b, S::kIdescPV, (q > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(bKVEmpty(slot));
-          tc_commit(bODone);
+          tc_commit(bODone(s_cnt + q));
           return true;
         };
         if (nch == 0) {
@@ -608,13 +629,11 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           s3 += sv[c + 3];
         }
         l = l * alpha + ((s0 + s1) + (s2 + s3));
-        if (q > 0) {
-          // O must hold PV_{q-1} before it is rescaled (S_q may finish first).
-          ok = __all_sync(0xffffffffu, ctl.wait(bODone, (sc - 1) & 1));
+        if (resc) {
+          // O must hold PV_{q-1} before it is rescaled; only rescaling chunks wait.
+          ok = __all_sync(0xffffffffu, ctl.wait(bODone(sc - 1), ((sc - 1) >> 1) & 1));
           if (!ok) break;
           tc_fence_after();
-        }
-        if (resc) {
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
             float ov[32];
@@ -639,7 +658,8 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       }
       if (!ok) break;
       if (nch > 0) {
-        ok = __all_sync(0xffffffffu, ctl.wait(bODone, (s_cnt + nch - 1) & 1));
+        const int last = s_cnt + nch - 1;
+        ok = __all_sync(0xffffffffu, ctl.wait(bODone(last), (last >> 1) & 1));
         if (!ok) break;
         tc_fence_after();
       }
@@ -808,9 +828,9 @@ int launch_forward(const ForwardArgs& a) {
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
   if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 4, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 8, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 4, 2>(a, p);
   if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 8, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 4, 2>(a, p);
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 
@@ -838,9 +858,9 @@ int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int3
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
   if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 4, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 8, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 4, 2>(a, p);
   if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 8, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 4, 2>(a, p);
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 

@@ -96,6 +96,58 @@ def test_non_default_scale():
     lay.close()
 
 
+@pytest.mark.parametrize("kind,n,B,L,heads,kv,d,pat", [
+    (OL.BAND_GLOBAL, 2048, 128, 1, 2, 2, 128, dict(window=10 ** 6, global_first=1)),
+    (OL.DYADIC, 4096 - 7, 64, 1, 4, 2, 128, dict(window=2, global_first=1, dyadic_kmin=2)),
+    (OL.RANDOM, 3072, 128, 2, 2, 2, 64, dict(density=0.4, seed=3)),
+])
+def test_rescale_path(kind, n, B, L, heads, kv, d, pat):
+    """Keys grow in magnitude along the sequence, so each later block's scores
+    exceed the running maximum by far more than the rescale threshold and the
+    kernel must rescale O (with N(0,1) inputs it essentially never does)."""
+    scale = default_scale(d)
+    lay = bsa.Layout(kind, n, B, L, torch.cuda.current_device(), **pat)
+    qb, kb, vb = inputs.qkv_bits(heads, kv, n, d, (5, 6, 7))
+    grow = np.repeat(1.0 + 0.8 * np.arange(-(-n // B)), B)[:n].astype(np.float32)
+    kf = inputs.bf16_bits_to_f32(kb) * grow[None, :, None]
+    qf = np.abs(inputs.bf16_bits_to_f32(qb))
+    kf = np.abs(kf)                      # positive scores that grow with the key block
+    kb = inputs.f32_to_bf16_bits(kf)
+    qb = inputs.f32_to_bf16_bits(qf * 0.5)
+    # halve V so |o| stays below 4, where bf16 output still resolves 1e-2
+    vb = inputs.f32_to_bf16_bits(inputs.bf16_bits_to_f32(vb) * 0.5)
+    from gpu_common import to_device_bf16
+    q, k, v = to_device_bf16(qb), to_device_bf16(kb), to_device_bf16(vb)
+    o, lse = bsa.attention(q, k, v, lay, scale)
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+    sets = OL.kept_sets(kind, n, B, L, **pat)
+    o_ref, lse_ref = _oracle((qb, kb, vb), sets, B, scale)
+    # row maxima span many multiples of the kernel's rescale threshold (8 in
+    # exp2 units, about 5.5 in lse units): the rescale path is really taken
+    assert float(np.nanmax(lse_ref) - np.nanmin(lse_ref[np.isfinite(lse_ref)])) > 40
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "rescale")
+    lay.close()
+
+
+def test_large_scale_rescales():
+    """A large softmax scale makes row maxima jump far beyond the rescale
+    threshold between blocks; V is halved so |o| stays where bf16 resolves 1e-2."""
+    n, B, d = 2048, 64, 128
+    pat = dict(window=2, global_first=1, dyadic_kmin=2)
+    lay = bsa.Layout(OL.DYADIC, n, B, 1, torch.cuda.current_device(), **pat)
+    qb, kb, vb = inputs.qkv_bits(4, 2, n, d)
+    vb = inputs.f32_to_bf16_bits(inputs.bf16_bits_to_f32(vb) * 0.5)
+    from gpu_common import to_device_bf16
+    o, lse = bsa.attention(to_device_bf16(qb), to_device_bf16(kb), to_device_bf16(vb), lay, 1.5)
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+    sets = OL.kept_sets(OL.DYADIC, n, B, 1, **pat)
+    o_ref, lse_ref = _oracle((qb, kb, vb), sets, B, 1.5)
+    assert_close(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref, "scale 1.5")
+    lay.close()
+
+
 # ----------------------------------------------------------------- full size
 FULL = ["band_global_32k", "bf1_dyadic_gqa_32k", "static_random_131k"]
 
