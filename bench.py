@@ -11,9 +11,10 @@ pinned host buffers (layout compile + H2D of q, k, v + forward + D2H of o and
 lse inside every timed step).
 
 ``python bench.py [--gpus N --steps K --warmup W] [--impl reference]``; under
-torchrun each rank runs an independent replica (the work items of this path
-share nothing, so there is no data-path collective) and rank 0 prints one JSON
-line with the max-over-ranks device time.
+torchrun the global batch is one problem of the workload per rank and each
+rank runs its own (the work items of this path share nothing, so there is no
+data-path collective); rank 0 prints one JSON line with the max-over-ranks
+device time and the whole-job throughput.
 """
 from __future__ import annotations
 
@@ -34,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from block_sparse_long_bsa_b200 import inputs as synth                  # noqa: E402
+from block_sparse_long_bsa_b200 import sharding                         # noqa: E402
 from block_sparse_long_bsa_b200.workloads import WORKLOADS, ORDER, HEADLINE  # noqa: E402
 
 METRIC = "block-sparse attn fwd effective TFLOPS (4·d·kept pairs/s), % of B200 bf16 peak"
@@ -109,23 +111,64 @@ def profiled_traffic(workload):
 
 
 class ClockSampler:
-    """nvidia-smi samples (SM clock, max clock, throttle reasons) in a thread."""
+    """SM clock, max clock, power and clock-event (throttle) reasons, sampled
+    in a thread during the run: through NVML every ``period_ms`` (the timed
+    region of a step is well under a millisecond, so the sampling is dense),
+    else through ``nvidia-smi -lms``.  Read-only: no setting is changed."""
 
-    def __init__(self, gpu_index: int, period_ms: int = 100):
-        self.cmd = ["nvidia-smi", "-i", str(gpu_index),
-                    "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
-                    "--format=csv,noheader,nounits", f"-lms", str(period_ms)]
+    def __init__(self, cuda_index: int, period_ms: float = 2.0):
+        self.cuda_index = cuda_index
+        self.period = period_ms / 1e3
         self.samples = []
         self.proc = None
         self.thread = None
+        self.stop_flag = threading.Event()
+        self.source = "none"
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            pr = torch.cuda.get_device_properties(self.cuda_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+            nv, h = self._nvml_handle()
+            max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            return self._start_smi()
+        self.source = "nvml"
+
+        def poll():
+            while not self.stop_flag.is_set():
+                try:
+                    mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1e3
+                    rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    self.samples.append((time.time(), mhz, max_mhz, pw, rs))
+                except Exception:
+                    pass
+                time.sleep(self.period)
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+
+    def _start_smi(self):
+        cmd = ["nvidia-smi", "-i", str(self.cuda_index),
+               "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+               "--format=csv,noheader,nounits", "-lms", "100"]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
         except OSError:
             self.proc = None
             return
+        self.source = "nvidia-smi"
+
         def reader():
             for line in self.proc.stdout:
                 parts = [p.strip() for p in line.split(",")]
@@ -140,6 +183,7 @@ class ClockSampler:
         self.thread.start()
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc:
             self.proc.terminate()
             try:
@@ -165,7 +209,7 @@ class ClockSampler:
         names = [nm for bit, nm in THROTTLE_BITS.items() if reasons & bit]
         return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": max(s[2] for s in win),
                 "reasons": names, "power_w_max": max(s[3] for s in win),
-                "samples": len(loaded), "window": note}
+                "samples": len(loaded), "window": note, "source": self.source}
 
 
 def threads_in_use():
@@ -250,10 +294,10 @@ def run_reference(args, w):
 
 
 def workload_config(w, gpus):
-    return {"workload": w.name, "batch": w.batch, "q_heads": w.q_heads,
+    return {"workload": w.name, "batch": w.batch, "global_batch": w.batch * gpus, "q_heads": w.q_heads,
             "kv_heads": w.kv_heads_per_seq, "n": w.n, "d": w.d, "B": w.B,
             "layout_heads": w.layout_heads, "pattern": w.description,
-            "parallelism": "replicas" if gpus == 1 else f"replicas x{gpus} (independent batches per GPU)",
+            "parallelism": f"dp{gpus} (one problem per GPU, no data-path collective)",
             "l2": "inputs exceed the 126 MB L2 and a 256 MiB buffer is written between timed steps"}
 
 
@@ -261,7 +305,7 @@ def workload_config(w, gpus):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=HEADLINE, choices=ORDER)
@@ -306,8 +350,12 @@ def main():
     row_ptr, col_idx = lay.csr()
     pairs, flops, compulsory = workload_work(w, row_ptr, col_idx)
 
-    # --- inputs (seeded, synthetic; resident in HBM for the device-timed value)
-    qb, kb, vb = synth.qkv_bits(w.heads, w.kv_heads, w.n, w.d)
+    # --- inputs (seeded, synthetic; resident in HBM for the device-timed value).
+    # The global batch is one problem of the workload per rank; rank r owns
+    # problem r and draws its inputs from that problem's seeds.
+    mine = sharding.shard(world, world, rank)
+    seeds = sharding.element_seeds(mine.start)
+    qb, kb, vb = synth.qkv_bits(w.heads, w.kv_heads, w.n, w.d, seeds)
 
     def to_dev(bits):
         return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
@@ -346,13 +394,9 @@ def main():
     bsa.bsa_get_status(lay.handle)
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     local_total_ms = float(sum(step_ms))
-    total_ms = local_total_ms
-    if world > 1:
-        t = torch.tensor([local_total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = sharding.max_over_ranks(local_total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    value = sharding.aggregate_rate(flops * args.steps, world, total_ms * 1e-3) / 1e12
     clocks = sampler.summary(wall0 - 0.05, wall1 + 0.05)
 
     if args.only_device:
@@ -403,12 +447,8 @@ def main():
     torch.cuda.synchronize()
     for l2 in keep:
         l2.close()
-    e2e_ms = e_start.elapsed_time(e_end)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops * args.e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = sharding.max_over_ranks(e_start.elapsed_time(e_end), world, dev)
+    e2e_value = sharding.aggregate_rate(flops * args.e2e_steps, world, e2e_ms * 1e-3) / 1e12
     layout_bytes = 4 * (len(row_ptr) + len(col_idx) + len(row_ptr) - 1)
     pairs, flops = int(pairs), int(flops)
     h2d = q.numel() * 2 + k.numel() * 2 + v.numel() * 2 + layout_bytes
@@ -451,7 +491,8 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic N(0,1) bf16 from numpy default_rng seeds 0/1/2 (q/k/v); layout seed 17",
+            "data": "synthetic N(0,1) bf16 from numpy default_rng, q/k/v seeds 3r/3r+1/3r+2 on rank r; "
+                    "layout seed 17",
             "config": workload_config(w, world),
             "frac_of_peak": value / world / peak,
             "layout_build_ms": layout_ms,
