@@ -17,14 +17,14 @@
 //                        causal mask of "bsbr", Solution; BF1 section 3.1)
 //   m' = max(m, rowmax S); P = exp2((S - m') * scale*log2 e) as bf16 into TMEM
 //   O += P V_j                 (tcgen05.mma with A = P read from TMEM)
-// then o = O / l (bf16, TMA store) and lse = (m + log2 l) * ln 2.
+// then o = O / l (bf16, stored row by row) and lse = (m + log2 l) * ln 2.
 // The running max is only moved when a block's max exceeds it by more than
 // 2^8 (in exp2 units), which keeps P <= 256 (exact in bf16's range) and skips
 // almost every rescale of O; the final normalisation uses the same max as the
 // sum, so the result is the plain softmax.
 //
-// Roles (192 threads): warp 0 issues TMA loads (Q once, then K_j and V_j into a
-// ring of shared-memory slots); warp 1 owns TMEM and issues the MMAs from one
+// Roles (192 threads): warp 0 issues TMA loads (Q once, then K_j and V_j into
+// two rings of shared-memory slots); warp 1 owns TMEM and issues the MMAs from one
 // thread; warps 2-5 do the softmax, one query row per thread (a warp can only
 // reach its own quarter of the TMEM lanes: warp w serves rows 32*(w%4) ..).
 // Every wait on an mbarrier is bounded; when one runs out the kernel records
@@ -140,13 +140,6 @@ __device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64_t 
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void named_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // TMA (no multicast anywhere in this library).
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -165,9 +158,37 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src,
                "r"(src), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
 }
-__device__ __forceinline__ void tma_store_commit_and_wait() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
+                                            int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+// One 64-key chunk of K or V (rows r0 .. r0+63 of head h, all d columns) as a
+// single box: the tensor map's third dimension walks the 64-column swizzle
+// atoms, so the box lands as [atom][row][64 columns], the layout the MMA
+// descriptors read.
+template <int HD>
+__device__ __forceinline__ void tma_load_kv(uint32_t dst, const CUtensorMap* m, uint32_t bar, int r0, int h) {
+  if constexpr (HD == 128) tma_load_4d(dst, m, bar, 0, r0, 0, h);
+  else tma_load_3d(dst, m, bar, 0, r0, h);
+}
+// The whole 128-row Q tile as a single box: for B = 64 the box spans two
+// consecutive heads (the two stacked query blocks), for B = 128 one block.
+template <int BLK, int HD>
+__device__ __forceinline__ void tma_load_q(uint32_t dst, const CUtensorMap* m, uint32_t bar, int r0, int h) {
+  if constexpr (HD == 128 && BLK == 64) tma_load_4d(dst, m, bar, 0, r0, h, 0);
+  else if constexpr (HD == 128) tma_load_4d(dst, m, bar, 0, r0, 0, h);
+  else tma_load_3d(dst, m, bar, 0, r0, h);
 }
 
 // tcgen05 / TMEM
@@ -268,11 +289,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-               : "memory");
-}
-
 // tcgen05 shared-memory matrix descriptor for a 128-byte-swizzled operand
 // (the layout TMA writes with CU_TENSOR_MAP_SWIZZLE_128B): start address,
 // leading and stride byte offsets (16-byte units), version 1, swizzle mode 2.
@@ -298,8 +314,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
 // B = 64, two for B = 128), so S is a 128 x 64 fp32 tile, two S buffers and the
 // O accumulator fit in 256 TMEM columns, and two CTAs share each SM.
 constexpr int kChunk = 64;
+constexpr int kKSlots = 2;   // K ring: K_c lives in slot c % 2
+constexpr int kVSlots = 3;   // V ring: V_c lives in slot c % 3
+constexpr int kODone = 3;    // PV_c completes o_done[c % 3]
 
-template <int BLK, int HD, int KVS>
+template <int BLK, int HD>
 struct KernelShape {
   static constexpr int kCPB = BLK / kChunk;                  // chunks per kept block
   static constexpr int kSubs = kTileM / BLK;                 // query blocks stacked in the tile
@@ -308,16 +327,17 @@ struct KernelShape {
   static constexpr int kTileBytes = kChunk * HD * 2;         // one 64-key chunk of K or V
   static constexpr int kAtomRowsQ = kTileM * 128;            // bytes of one Q atom column
   static constexpr int kAtomRowsKV = kChunk * 128;           // bytes of one K/V atom column
+  static constexpr int kOffK = kQBytes;
+  static constexpr int kOffV = kOffK + kKSlots * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
+  // barriers: q_full, q_free, k_full[2], v_full[3], s_full[2], p_full[2],
+  //           o_done[3], o_free, drain, never, stage_free
+  static constexpr int kNumBars = 2 + kKSlots + kVSlots + 2 + 2 + kODone + 4;
   static constexpr int kWarpStage = 32 * 128;                // one warp's 32 rows x 64 columns of o
-  static constexpr int kOffKV = kQBytes;
-  static constexpr int kOffStage = kOffKV + KVS * kTileBytes;
-  static constexpr int kOffBar = kOffStage + 4 * kWarpStage;
-  // barriers: q_full, q_free, kv_full[KVS], s_full[2], p_full[2],
-  //           o_done[2] (PV products with even / odd index), o_free, drain, never
-  static constexpr int kNumBars = 2 + KVS + 4 + 5;
+  static_assert(4 * (HD / 64) * kWarpStage == 2 * kTileBytes, "o staging fills two V slots");
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kOffHist = kOffMisc + 16;             // producer's ring history [KVS] int
-  static constexpr int kSmemUsed = kOffHist + 4 * KVS;
+  static constexpr int kOffPend = kOffMisc + 16;             // producer's pending-staging FIFO
+  static constexpr int kSmemUsed = kOffPend + 32;
   static constexpr int kColS = 0;                            // S buffers: columns 0..63, 64..127
   static constexpr int kColO = 2 * kChunk;
   static constexpr uint32_t kTmemCols = 256;
@@ -326,7 +346,6 @@ struct KernelShape {
   static_assert(2 * kChunk + HD <= 256, "TMEM budget");
   static_assert(BLK == 64 || BLK == 128, "block size");
   static_assert(HD == 64 || HD == 128, "head dim");
-  static_assert(KVS == 4, "the ring-slot hand-off relies on exactly four slots");
 };
 
 // One work item = (head group, rank in its layout head's longest-first order).
@@ -358,12 +377,26 @@ __device__ __forceinline__ int item_at(int k) {
   return k * G + ((k & 1) ? (G - 1 - c) : c);
 }
 
-template <int BLK, int HD, int KVS, int MIN_CTAS>
+__device__ __forceinline__ void st_global_v4(void* ptr, const uint32_t* u) {
+  asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(ptr), "r"(u[0]), "r"(u[1]), "r"(u[2]),
+               "r"(u[3])
+               : "memory");
+}
+
+// Chunk c (counted over all items of the CTA) uses S buffer c & 1, K slot
+// c % 2 and V slot c % 3.  MMAs are issued in the order QK_0, QK_1, PV_0,
+// QK_2, PV_1, ..., and the producer loads in the same order (K_{q+1} before
+// V_q).  A K slot frees when QK_{c-2} completes (s_full of that buffer), a V
+// slot when PV_{c-3} completes (o_done[c % 3]).  Each such barrier completes
+// once per product of its residue class, and the load that waits on it is
+// the one the next product of that class needs, so a parity wait can be
+// neither one phase early nor two phases late.
+template <int BLK, int HD, int MIN_CTAS>
 __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                    const Params p) {
-  using S = KernelShape<BLK, HD, KVS>;
+  using S = KernelShape<BLK, HD>;
   constexpr int CPB = S::kCPB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_addr(smem_raw);
@@ -376,26 +409,35 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   uint8_t* gbase = smem_raw;
 
   const uint32_t sQ = base;
-  const uint32_t sKV = base + S::kOffKV;
-  const uint32_t sStage = base + S::kOffStage;
+  const uint32_t sK = base + S::kOffK;
+  const uint32_t sV = base + S::kOffV;
   const uint32_t bar0 = base + S::kOffBar;
   const uint32_t bQFull = bar0;
   const uint32_t bQFree = bar0 + 8u;
-  auto bKVFull = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto bSFull = [&](int s) { return bar0 + 8u * (2 + KVS + s); };
-  auto bPFull = [&](int s) { return bar0 + 8u * (2 + KVS + 2 + s); };
-  // PV product j completes barrier o_done[j & 1]: each barrier then advances
-  // once per two products, so a softmax warp that skips waiting on some of
-  // them is never two phases behind when it does wait (S_q is committed after
-  // PV_{q-2}, and PV_{q+1} cannot finish before P_{q+1} exists).
-  const uint32_t bODone0 = bar0 + 8u * (2 + KVS + 4);
-  auto bODone = [&](int j) { return bODone0 + 8u * (j & 1); };
-  const uint32_t bOFree = bODone0 + 16u;
-  const uint32_t bDrain = bODone0 + 24u;
-  const uint32_t bNever = bODone0 + 32u;
+  const uint32_t bKFull0 = bar0 + 16u;
+  const uint32_t bVFull0 = bKFull0 + 8u * kKSlots;
+  const uint32_t bSFull0 = bVFull0 + 8u * kVSlots;
+  const uint32_t bPFull0 = bSFull0 + 16u;
+  const uint32_t bODone0 = bPFull0 + 16u;
+  const uint32_t bOFree = bODone0 + 8u * kODone;
+  const uint32_t bDrain = bOFree + 8u;
+  const uint32_t bNever = bOFree + 16u;
+  // The epilogue of an item stages o in the V slots of its last two chunks
+  // (free once its last PV is done); stage_free completes when the TMA stores
+  // out of them have read them, once per item with at least one chunk.
+  const uint32_t bStageFree = bOFree + 24u;
+  auto bKFull = [&](int c) { return bKFull0 + 8u * (c % kKSlots); };
+  auto bVFull = [&](int c) { return bVFull0 + 8u * (c % kVSlots); };
+  auto bSFull = [&](int c) { return bSFull0 + 8u * (c & 1); };
+  auto bPFull = [&](int c) { return bPFull0 + 8u * (c & 1); };
+  auto bODone = [&](int c) { return bODone0 + 8u * (c % kODone); };
+  // phase parities of chunk c's barriers
+  auto parK = [](int c) { return uint32_t(c / kKSlots) & 1u; };
+  auto parV = [](int c) { return uint32_t(c / kVSlots) & 1u; };
+  auto parS = [](int c) { return uint32_t(c >> 1) & 1u; };
+  auto parO = [](int c) { return uint32_t(c / kODone) & 1u; };
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(gbase + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + S::kOffMisc + 4);
-  int* ring_hist = reinterpret_cast<int*>(gbase + S::kOffHist);   // chunk index | (is V) << 31
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -406,16 +448,17 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   if (threadIdx.x == 0) {
     mbar_init(bQFull, 1);
     mbar_init(bQFree, 1);
-    for (int s = 0; s < KVS; ++s) mbar_init(bKVFull(s), 1);
+    for (int s = 0; s < kKSlots; ++s) mbar_init(bKFull0 + 8u * s, 1);
+    for (int s = 0; s < kVSlots; ++s) mbar_init(bVFull0 + 8u * s, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bSFull(s), 1);
-      mbar_init(bPFull(s), 128);
+      mbar_init(bSFull0 + 8u * s, 1);
+      mbar_init(bPFull0 + 8u * s, 128);
     }
-    mbar_init(bODone(0), 1);
-    mbar_init(bODone(1), 1);
+    for (int s = 0; s < kODone; ++s) mbar_init(bODone0 + 8u * s, 1);
     mbar_init(bOFree, 128);
     mbar_init(bDrain, 1);
     mbar_init(bNever, 1);
+    mbar_init(bStageFree, 4);
     *abort_flag = 0;
     fence_barrier_init();
     if (!p.debug_never) {
@@ -437,9 +480,14 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   if (warp == 0) {
     // ================================================================ producer
     if (lane == 0) {
-      int issued = 0;        // K/V chunk loads issued so far (ring position)
-      int q_loads = 0;       // Q tile loads issued so far
-      int chunks = 0;        // chunks of earlier items (global chunk index base)
+      int kc = 0;            // K chunk loads issued (global chunk index of the next one)
+      int vc = 0;            // V chunk loads issued
+      int q_loads = 0;       // Q tile loads issued
+      // Items with chunks whose staging slots the producer has not yet seen
+      // freed: (ordinal among items with chunks, global index of last chunk).
+      int* pend_ord = reinterpret_cast<int*>(gbase + S::kOffPend);
+      int* pend_last = pend_ord + 4;
+      int pend_head = 0, pend_tail = 0, n_nonempty = 0;
       bool ok = true;
       if (p.debug_never) ok = ctl.wait(bNever, 0);
       for (int k = 0; ok; ++k) {
@@ -449,52 +497,59 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         // the previous item's last QK^T has finished reading the Q buffer
         if (k > 0 && !(ok = ctl.wait(bQFree, (k - 1) & 1))) break;
         mbar_expect_tx(bQFull, S::kQBytes);
-        for (int sub = 0; sub < S::kSubs; ++sub)
-          for (int a = 0; a < S::kAtoms; ++a)
-            tma_load_3d(sQ + a * S::kAtomRowsQ + sub * BLK * 128, &tmQ, bQFull, a * 64,
-                        it.row * BLK, it.h0 + (p.pack == 2 ? sub : 0));
+        // For B = 64 without a partner head the second block of the tile is
+        // the next head's (or zeros past the last head): its rows are discarded.
+        tma_load_q<BLK, HD>(sQ, &tmQ, bQFull, it.row * BLK, it.h0);
         ++q_loads;
-        // Chunk q of the item owns ring positions 2q (K) and 2q + 1 (V) after
-        // the item's base, so every chunk occupies exactly two positions.
         const int nch = it.len * CPB;
-        for (int idx = 0; idx < 2 * nch && ok; ++idx) {
-          const int q = idx >> 1;
-          const bool is_v = idx & 1;
-          const int key0 = __ldg(p.col_idx + it.start + q / CPB) * BLK + (q % CPB) * kChunk;
-          const int l = issued, slot = l % KVS;
-          if (l >= KVS) {
-            // The slot frees when the product that read its previous tile is
-            // done: QK^T of that chunk for a K tile (s_full), PV for a V tile
-            // (o_done).  A slot holds chunk c, then chunk c + 2 of the same
-            // kind, so with four slots the next completion of the same
-            // barrier needs the very tile loaded here and the phase test can
-            // be neither behind nor ahead by two phases.
-            const int prev = ring_hist[slot];
-            const int pc = prev & 0x7fffffff;
-            const uint32_t bar = (prev < 0) ? bODone(pc) : bSFull(pc & 1);
-            if (!(ok = ctl.wait(bar, (pc >> 1) & 1))) break;
-          }
-          ring_hist[slot] = (is_v ? int(0x80000000u) : 0) | (chunks + q);
-          mbar_expect_tx(bKVFull(slot), S::kTileBytes);
-          const CUtensorMap* m = is_v ? &tmV : &tmK;
-          for (int a = 0; a < S::kAtoms; ++a)
-            tma_load_3d(sKV + slot * S::kTileBytes + a * S::kAtomRowsKV, m, bKVFull(slot), a * 64, key0,
-                        it.kvh);
-          ++issued;
+        if (nch > 0) {
+          pend_ord[pend_tail & 3] = n_nonempty++;
+          pend_last[pend_tail & 3] = kc + nch - 1;
+          ++pend_tail;
         }
-        chunks += nch;
+        auto key0 = [&](int q) { return __ldg(p.col_idx + it.start + q / CPB) * BLK + (q % CPB) * kChunk; };
+        auto load_k = [&](int q) -> bool {
+          const int c = kc;
+          if (c >= kKSlots && !ctl.wait(bSFull(c), parS(c - kKSlots))) return false;
+          const uint32_t dst = sK + (c % kKSlots) * S::kTileBytes;
+          mbar_expect_tx(bKFull(c), S::kTileBytes);
+          const int r0 = key0(q);
+          tma_load_kv<HD>(dst, &tmK, bKFull(c), r0, it.kvh);
+          ++kc;
+          return true;
+        };
+        auto load_v = [&](int q) -> bool {
+          const int c = vc;
+          if (c >= kVSlots && !ctl.wait(bODone(c), parO(c - kVSlots))) return false;
+          // V_c refills the slot of chunk c - 3; if that chunk or chunk c - 2
+          // was the last of an item, its epilogue staged o there.
+          while (pend_head != pend_tail && c >= pend_last[pend_head & 3] + 2) {
+            if (!ctl.wait(bStageFree, uint32_t(pend_ord[pend_head & 3]) & 1u)) return false;
+            ++pend_head;
+          }
+          const uint32_t dst = sV + (c % kVSlots) * S::kTileBytes;
+          mbar_expect_tx(bVFull(c), S::kTileBytes);
+          const int r0 = key0(q);
+          tma_load_kv<HD>(dst, &tmV, bVFull(c), r0, it.kvh);
+          ++vc;
+          return true;
+        };
+        if (nch > 0) ok = load_k(0);
+        for (int q = 0; q < nch && ok; ++q) {
+          if (q + 1 < nch) ok = load_k(q + 1);
+          if (ok) ok = load_v(q);
+        }
       }
       // Never leave the CTA with copies in flight into its shared memory.
       if (q_loads > 0) wait_drain(bQFull, (q_loads - 1) & 1, 200000000ull);
-      for (int l = (issued > KVS ? issued - KVS : 0); l < issued; ++l)
-        wait_drain(bKVFull(l % KVS), (l / KVS) & 1, 200000000ull);
+      for (int c = (kc > kKSlots ? kc - kKSlots : 0); c < kc; ++c) wait_drain(bKFull(c), parK(c), 200000000ull);
+      for (int c = (vc > kVSlots ? vc - kVSlots : 0); c < vc; ++c) wait_drain(bVFull(c), parV(c), 200000000ull);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       bool ok = true;
-      int kv = 0;            // K/V chunks consumed (ring position)
-      int s_cnt = 0;         // QK^T products issued (S buffer rotation)
+      int c0 = 0;            // chunks of earlier items (global chunk index base)
       if (p.debug_never) ok = ctl.wait(bNever, 0);
       for (int k = 0; ok; ++k) {
         const int t = item_at(k);
@@ -503,46 +558,41 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         const int nch = it.len * CPB;
         if (!(ok = ctl.wait(bQFull, k & 1))) break;
         tc_fence_after();
-        // ring positions of K_q and V_q
-        auto k_pos = [&](int q) { return kv + 2 * q; };
-        auto v_pos = [&](int q) { return kv + 2 * q + 1; };
         auto issue_qk = [&](int q) -> bool {
-          const int l = k_pos(q), slot = l % KVS;
-          if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
+          const int c = c0 + q;
+          if (!ctl.wait(bKFull(c), parK(c))) return false;
           tc_fence_after();
-          const int sb = (s_cnt + q) & 1;
-          const uint32_t d = tmem + S::kColS + sb * kChunk;
-          const uint32_t kb = sKV + slot * S::kTileBytes;
+          const uint32_t d = tmem + S::kColS + (c & 1) * kChunk;
+          const uint32_t kb = sK + (c % kKSlots) * S::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint64_t a = sw128_desc(sQ + (kk >> 2) * S::kAtomRowsQ + (kk & 3) * 32, 16, 1024);
             const uint64_t b = sw128_desc(kb + (kk >> 2) * S::kAtomRowsKV + (kk & 3) * 32, 16, 1024);
             mma_ss(d, a, b, S::kIdescQK, kk > 0 ? 1u : 0u);
           }
-          tc_commit(bSFull(sb));
+          tc_commit(bSFull(c));
           if (q == nch - 1) tc_commit(bQFree);      // last reader of this Q tile
           return true;
         };
         auto issue_pv = [&](int q) -> bool {
-          const int sc = s_cnt + q, sb = sc & 1;
-          if (!ctl.wait(bPFull(sb), (sc >> 1) & 1)) return false;
+          const int c = c0 + q;
+          if (!ctl.wait(bPFull(c), parS(c))) return false;
           tc_fence_after();
           if (q == 0 && k > 0) {
             // the previous item's epilogue has read O out of TMEM
             if (!ctl.wait(bOFree, (k - 1) & 1)) return false;
             tc_fence_after();
           }
-          const int l = v_pos(q), slot = l % KVS;
-          if (!ctl.wait(bKVFull(slot), (l / KVS) & 1)) return false;
+          if (!ctl.wait(bVFull(c), parV(c))) return false;
           tc_fence_after();
-          const uint32_t pa = tmem + S::kColS + sb * kChunk;
-          const uint32_t vb = sKV + slot * S::kTileBytes;
+          const uint32_t pa = tmem + S::kColS + (c & 1) * kChunk;
+          const uint32_t vb = sV + (c % kVSlots) * S::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < kChunk / 16; ++kk) {
             const uint64_t b = sw128_desc(vb + kk * 16 * 128, S::kAtomRowsKV, 1024);
             mma_ts(tmem + S::kColO, pa + kk * 8, b, S::kIdescPV, (q > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(bODone(s_cnt + q));
+          tc_commit(bODone(c));
           return true;
         };
         if (nch == 0) {
@@ -556,8 +606,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             if (ok) ok = issue_pv(q);
           }
         }
-        kv += 2 * nch;
-        s_cnt += nch;
+        c0 += nch;
       }
       // Wait for every MMA this thread issued before TMEM can be released.
       tc_commit(bDrain);
@@ -570,11 +619,23 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     const int sub = r / BLK;
     const int rl = r - sub * BLK;            // row inside its query block
     const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
-    const uint32_t stage = sStage + q4 * S::kWarpStage;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    int s_cnt = 0;                           // chunks seen (S buffer rotation, o_done phase)
-    bool stores_pending = false;
+    int s_cnt = 0;                           // chunks seen (global chunk index base)
+    bool stage_pending = false;              // this warp's last staging stores not yet released
+    // Once the TMA stores of the previous epilogue have read the staging box,
+    // tell the producer (one arrival per warp); deferred so the store drains
+    // while this warp already works on the next item.
+    auto release_stage = [&]() {
+      if (stage_pending) {
+        if (lane == 0) {
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          mbar_arrive(bStageFree);
+        }
+        __syncwarp();
+        stage_pending = false;
+      }
+    };
     if (p.debug_never) ok = __all_sync(0xffffffffu, ctl.wait(bNever, 0));
     for (int k = 0; ok; ++k) {
       const int t = item_at(k);
@@ -582,12 +643,14 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       const Item it = decode_item(p, t);
       const int nch = it.len * CPB;
       const int diag_first = it.diag_last ? nch - CPB : nch;   // first chunk of the diagonal block
+      if (nch == 0) release_stage();
       float m2 = -INFINITY;                  // running max, in exp2 units
       float l = 0.f;                         // running sum of P
       for (int q = 0; ok && q < nch; ++q) {
         const int sc = s_cnt + q, s = sc & 1;
-        ok = __all_sync(0xffffffffu, ctl.wait(bSFull(s), (sc >> 1) & 1));
+        ok = __all_sync(0xffffffffu, ctl.wait(bSFull(sc), parS(sc)));
         if (!ok) break;
+        if (q == 0) release_stage();
         tc_fence_after();
         float sv[kChunk];
         tmem_ld32(lane_base + S::kColS + s * kChunk, sv);
@@ -630,8 +693,8 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         }
         l = l * alpha + ((s0 + s1) + (s2 + s3));
         if (resc) {
-          // O must hold PV_{q-1} before it is rescaled; only rescaling chunks wait.
-          ok = __all_sync(0xffffffffu, ctl.wait(bODone(sc - 1), ((sc - 1) >> 1) & 1));
+          // O must hold PV_{sc-1} before it is rescaled; only rescaling chunks wait.
+          ok = __all_sync(0xffffffffu, ctl.wait(bODone(sc - 1), parO(sc - 1)));
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -653,67 +716,73 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bPFull(s));
+        mbar_arrive(bPFull(sc));
         m2 = m_new;
       }
       if (!ok) break;
       if (nch > 0) {
         const int last = s_cnt + nch - 1;
-        ok = __all_sync(0xffffffffu, ctl.wait(bODone(last), (last >> 1) & 1));
+        ok = __all_sync(0xffffffffu, ctl.wait(bODone(last), parO(last)));
         if (!ok) break;
         tc_fence_after();
       }
-      // ---- epilogue: o = O / l, 64 columns at a time through this warp's
-      // 32-row staging box and a TMA store; lse straight to global
-      const int r0 = q4 * 32;                // first row of this warp
-      const int sub0 = r0 / BLK;
-      const int tok0 = it.row * BLK + (r0 - sub0 * BLK);
-      const int head0 = it.h0 + (p.pack == 2 ? sub0 : 0);
-      const bool warp_stores = sub0 < p.pack;
+      // ---- epilogue: o = O / l as bf16 through this warp's 32-row staging box
+      // in a V slot of the item's last two chunks and a TMA store (o rows past
+      // n are clipped by the store); lse straight to global
+      const int tok = it.row * BLK + rl;
+      const int head = it.h0 + (p.pack == 2 ? sub : 0);
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      if (nch > 0) {
+        const int last = s_cnt + nch - 1;
+        const int r0 = q4 * 32;              // first row of this warp
+        const int sub0 = r0 / BLK;
+        const int tok0 = it.row * BLK + (r0 - sub0 * BLK);
+        const int head0 = it.h0 + (p.pack == 2 ? sub0 : 0);
+        const bool warp_stores = sub0 < p.pack;
 #pragma unroll
-      for (int a = 0; a < S::kAtoms; ++a) {
-        float ov[64];
-        if (nch > 0) {
+        for (int a = 0; a < S::kAtoms; ++a) {
+          float ov[64];
           tmem_ld32(lane_base + S::kColO + a * 64, ov);
           tmem_ld32(lane_base + S::kColO + a * 64 + 32, ov + 32);
           tmem_wait_ld();
-        } else {
+          if (a == S::kAtoms - 1) {
+            // O has been read: the next item's first PV may overwrite it
+            tc_fence_before();
+            mbar_arrive(bOFree);
+          }
+          // the two slots as one 2 x tile area: warp q4, atom a at (q4 * atoms + a) boxes
+          const int off = (q4 * S::kAtoms + a) * S::kWarpStage;
+          const int j = off / S::kTileBytes;                       // 0: chunk last, 1: chunk last - 1
+          const uint32_t stage = sV + ((last - j + kVSlots) % kVSlots) * S::kTileBytes + off % S::kTileBytes;
 #pragma unroll
-          for (int e = 0; e < 64; ++e) ov[e] = 0.f;
-        }
-        if (a == S::kAtoms - 1) {
-          // O has been read: the next item's first PV may overwrite it
-          tc_fence_before();
-          mbar_arrive(bOFree);
-        }
-        if (stores_pending) {
-          // the previous store out of this staging box must have read it
-          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(stage + lane * 128 + ((ch ^ (lane & 7)) << 4),
+                         pack_bf16(ov[8 * ch] * inv, ov[8 * ch + 1] * inv),
+                         pack_bf16(ov[8 * ch + 2] * inv, ov[8 * ch + 3] * inv),
+                         pack_bf16(ov[8 * ch + 4] * inv, ov[8 * ch + 5] * inv),
+                         pack_bf16(ov[8 * ch + 6] * inv, ov[8 * ch + 7] * inv));
+          fence_proxy_async();
           __syncwarp();
-          stores_pending = false;
+          if (warp_stores && lane == 0 && !*abort_flag) tma_store_3d(&tmO, stage, a * 64, tok0, head0);
         }
+        if (lane == 0) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        stage_pending = true;
+      } else {
+        // an item without kept blocks: o = 0 (rare; plain stores)
+        if (sub < p.pack && tok < p.n && !*abort_flag) {
+          uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + (size_t(head) * p.n + tok) * HD * 2;
+          const uint32_t z[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(stage + lane * 128 + ((ch ^ (lane & 7)) << 4),
-                       pack_bf16(ov[8 * ch] * inv, ov[8 * ch + 1] * inv),
-                       pack_bf16(ov[8 * ch + 2] * inv, ov[8 * ch + 3] * inv),
-                       pack_bf16(ov[8 * ch + 4] * inv, ov[8 * ch + 5] * inv),
-                       pack_bf16(ov[8 * ch + 6] * inv, ov[8 * ch + 7] * inv));
-        fence_proxy_async();
-        __syncwarp();
-        if (warp_stores && lane == 0 && !*abort_flag) {
-          tma_store_3d(&tmO, stage, a * 64, tok0, head0);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          for (int w4 = 0; w4 < HD / 8; ++w4) st_global_v4(orow + w4 * 16, z);
         }
-        stores_pending = true;
+        tc_fence_before();
+        mbar_arrive(bOFree);
       }
-      const int tok = it.row * BLK + rl;
       if (sub < p.pack && tok < p.n)
-        p.lse[size_t(it.h0 + (p.pack == 2 ? sub : 0)) * p.n + tok] =
-            l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
+        p.lse[size_t(head) * p.n + tok] = l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
       s_cnt += nch;
     }
+    release_stage();
     if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     __syncwarp();
   }
@@ -753,23 +822,68 @@ int get_encoder() {
   return BSA_OK;
 }
 
-// [slices][n][d] bf16, box of 64 columns x rows x 1 slice, 128-byte swizzle.
-int encode_map(CUtensorMap* m, const void* ptr, int slices, int n, int d, int rows) {
-  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(slices)};
-  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(n) * cuuint64_t(d) * 2};
-  cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+int encode_tiled(CUtensorMap* m, const void* ptr, cuuint32_t rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box) {
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
   return BSA_OK;
 }
 
-template <int BLK, int HD, int KVS, int MIN_CTAS>
+// K or V [slices][n][d]: a 64-row chunk of one slice per box.  For d = 128 the
+// view is (column within atom, row, atom, slice), the atom dimension striding
+// 128 bytes, so one box holds both atoms.
+int encode_kv(CUtensorMap* m, const void* ptr, int slices, int n, int d) {
+  const cuuint64_t row = cuuint64_t(d) * 2, slice = cuuint64_t(n) * row;
+  if (d == 128) {
+    const cuuint64_t dims[4] = {64, cuuint64_t(n), 2, cuuint64_t(slices)};
+    const cuuint64_t str[3] = {row, 128, slice};
+    const cuuint32_t box[4] = {64, 64, 2, 1};
+    return encode_tiled(m, ptr, 4, dims, str, box);
+  }
+  const cuuint64_t dims[3] = {64, cuuint64_t(n), cuuint64_t(slices)};
+  const cuuint64_t str[2] = {row, slice};
+  const cuuint32_t box[3] = {64, 64, 1};
+  return encode_tiled(m, ptr, 3, dims, str, box);
+}
+
+// o [heads][n][d]: one warp's 32 rows x 64 columns per store box.
+int encode_o(CUtensorMap* m, const void* ptr, int heads, int n, int d) {
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(heads)};
+  const cuuint64_t str[2] = {cuuint64_t(d) * 2, cuuint64_t(n) * cuuint64_t(d) * 2};
+  const cuuint32_t box[3] = {64, 32, 1};
+  return encode_tiled(m, ptr, 3, dims, str, box);
+}
+
+// Q [heads][n][d]: one 128-row tile per box.  B = 128: one block of one head;
+// B = 64: the same block of two consecutive heads, the head dimension inside
+// the atom dimension so the box lands as [atom][head][row][64 columns].
+int encode_q(CUtensorMap* m, const void* ptr, int heads, int n, int d, int blk) {
+  const cuuint64_t row = cuuint64_t(d) * 2, slice = cuuint64_t(n) * row;
+  if (d == 128 && blk == 64) {
+    const cuuint64_t dims[4] = {64, cuuint64_t(n), cuuint64_t(heads), 2};
+    const cuuint64_t str[3] = {row, slice, 128};
+    const cuuint32_t box[4] = {64, 64, 2, 2};
+    return encode_tiled(m, ptr, 4, dims, str, box);
+  }
+  if (d == 128) {
+    const cuuint64_t dims[4] = {64, cuuint64_t(n), 2, cuuint64_t(heads)};
+    const cuuint64_t str[3] = {row, 128, slice};
+    const cuuint32_t box[4] = {64, 128, 2, 1};
+    return encode_tiled(m, ptr, 4, dims, str, box);
+  }
+  const cuuint64_t dims[3] = {64, cuuint64_t(n), cuuint64_t(heads)};
+  const cuuint64_t str[2] = {row, slice};
+  const cuuint32_t box[3] = {64, cuuint32_t(blk), cuuint32_t(blk == 64 ? 2 : 1)};
+  return encode_tiled(m, ptr, 3, dims, str, box);
+}
+
+template <int BLK, int HD, int MIN_CTAS>
 int launch_instance(const ForwardArgs& a, dev::Params p) {
-  using S = dev::KernelShape<BLK, HD, KVS>;
-  auto kern = dev::bsa_fwd_kernel<BLK, HD, KVS, MIN_CTAS>;
+  using S = dev::KernelShape<BLK, HD>;
+  auto kern = dev::bsa_fwd_kernel<BLK, HD, MIN_CTAS>;
   // Ask for enough shared memory that no more than MIN_CTAS CTAs share an SM,
   // so every resident CTA's TMEM allocation succeeds at once.
   int smem = S::kSmemUsed;
@@ -782,16 +896,16 @@ int launch_instance(const ForwardArgs& a, dev::Params p) {
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
   if (e != cudaSuccess || sms < 1) return set_error(BSA_ERR_CUDA, "cannot query the SM count");
   CUtensorMap mq, mk, mv, mo;
+  std::memset(&mo, 0, sizeof(mo));
   std::memset(&mq, 0, sizeof(mq));
   std::memset(&mk, 0, sizeof(mk));
   std::memset(&mv, 0, sizeof(mv));
-  std::memset(&mo, 0, sizeof(mo));
   int grid;
   if (!a.debug_never) {
-    int st = encode_map(&mq, a.q, a.heads, a.n, HD, BLK);
-    if (st == BSA_OK) st = encode_map(&mk, a.k, a.kv_heads, a.n, HD, dev::kChunk);
-    if (st == BSA_OK) st = encode_map(&mv, a.v, a.kv_heads, a.n, HD, dev::kChunk);
-    if (st == BSA_OK) st = encode_map(&mo, a.o, a.heads, a.n, HD, 32);
+    int st = encode_q(&mq, a.q, a.heads, a.n, HD, BLK);
+    if (st == BSA_OK) st = encode_kv(&mk, a.k, a.kv_heads, a.n, HD);
+    if (st == BSA_OK) st = encode_kv(&mv, a.v, a.kv_heads, a.n, HD);
+    if (st == BSA_OK) st = encode_o(&mo, a.o, a.heads, a.n, HD);
     if (st != BSA_OK) return st;
     grid = p.items < sms * MIN_CTAS ? p.items : sms * MIN_CTAS;
   } else {
@@ -827,10 +941,10 @@ int launch_forward(const ForwardArgs& a) {
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
-  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 4, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 4, 2>(a, p);
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 2>(a, p);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2>(a, p);
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 
@@ -857,10 +971,10 @@ int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int3
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
-  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 4, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 4, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 4, 2>(a, p);
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 2>(a, p);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2>(a, p);
   return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
 }
 
