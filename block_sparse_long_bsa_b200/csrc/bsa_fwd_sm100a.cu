@@ -59,6 +59,7 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   uint32_t* status;
+  uint32_t* work_counter;   // next unclaimed item of the longest-first list (zeroed before launch)
   int n, nb, heads, L, group;
   int items;         // work items in the longest-first list
   int pack;          // distinct heads per tile (1 or 2)
@@ -317,6 +318,7 @@ constexpr int kChunk = 64;
 constexpr int kKSlots = 2;   // K ring: K_c lives in slot c % 2
 constexpr int kVSlots = 3;   // V ring: V_c lives in slot c % 3
 constexpr int kODone = 3;    // PV_c completes o_done[c % 3]
+constexpr int kItemSlots = 8;  // items claimed by the producer, handed to the other roles
 
 template <int BLK, int HD>
 struct KernelShape {
@@ -331,13 +333,14 @@ struct KernelShape {
   static constexpr int kOffV = kOffK + kKSlots * kTileBytes;
   static constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
   // barriers: q_full, q_free, k_full[2], v_full[3], s_full[2], p_full[2],
-  //           o_done[3], o_free, drain, never, stage_free
-  static constexpr int kNumBars = 2 + kKSlots + kVSlots + 2 + 2 + kODone + 4;
+  //           o_done[3], o_free, drain, never, stage_free, item_full[8]
+  static constexpr int kNumBars = 2 + kKSlots + kVSlots + 2 + 2 + kODone + 4 + kItemSlots;
   static constexpr int kWarpStage = 32 * 128;                // one warp's 32 rows x 64 columns of o
   static_assert(4 * (HD / 64) * kWarpStage == 2 * kTileBytes, "o staging fills two V slots");
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffPend = kOffMisc + 16;             // producer's pending-staging FIFO
-  static constexpr int kSmemUsed = kOffPend + 32;
+  static constexpr int kOffItems = kOffPend + 32;            // claimed item indices, ring of 8
+  static constexpr int kSmemUsed = kOffItems + 4 * kItemSlots;
   static constexpr int kColS = 0;                            // S buffers: columns 0..63, 64..127
   static constexpr int kColO = 2 * kChunk;
   static constexpr uint32_t kTmemCols = 256;
@@ -369,12 +372,15 @@ __device__ __forceinline__ Item decode_item(const Params& p, int t) {
   return it;
 }
 
-// Persistent schedule: CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... of the
-// longest-first list (alternating direction each round keeps the per-CTA
-// totals even when lengths fall along the list).
-__device__ __forceinline__ int item_at(int k) {
-  const int G = gridDim.x, c = blockIdx.x;
-  return k * G + ((k & 1) ? (G - 1 - c) : c);
+// Persistent schedule: the producer of each CTA claims the next unclaimed
+// item of the longest-first list with one atomic add (greedy list
+// scheduling, so every CTA ends within about one item of the others) and
+// hands its index to the MMA and softmax roles through a ring of slots in
+// shared memory; -1 ends the stream.
+__device__ __forceinline__ int claim_item(const Params& p, int n_items) {
+  if (n_items <= 0) return -1;
+  const int t = int(atomicAdd(p.work_counter, 1u));
+  return t < n_items ? t : -1;
 }
 
 __device__ __forceinline__ void st_global_v4(void* ptr, const uint32_t* u) {
@@ -426,6 +432,9 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   // (free once its last PV is done); stage_free completes when the TMA stores
   // out of them have read them, once per item with at least one chunk.
   const uint32_t bStageFree = bOFree + 24u;
+  const uint32_t bItemFull0 = bOFree + 32u;
+  auto bItemFull = [&](int k) { return bItemFull0 + 8u * (k % kItemSlots); };
+  volatile int* item_slot = reinterpret_cast<volatile int*>(gbase + S::kOffItems);
   auto bKFull = [&](int c) { return bKFull0 + 8u * (c % kKSlots); };
   auto bVFull = [&](int c) { return bVFull0 + 8u * (c % kVSlots); };
   auto bSFull = [&](int c) { return bSFull0 + 8u * (c & 1); };
@@ -459,6 +468,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     mbar_init(bDrain, 1);
     mbar_init(bNever, 1);
     mbar_init(bStageFree, 4);
+    for (int s = 0; s < kItemSlots; ++s) mbar_init(bItemFull0 + 8u * s, 1);
     *abort_flag = 0;
     fence_barrier_init();
     if (!p.debug_never) {
@@ -490,9 +500,13 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       int pend_head = 0, pend_tail = 0, n_nonempty = 0;
       bool ok = true;
       if (p.debug_never) ok = ctl.wait(bNever, 0);
+      int next_t = ok ? claim_item(p, n_items) : -1;
       for (int k = 0; ok; ++k) {
-        const int t = item_at(k);
-        if (t >= n_items) break;
+        const int t = next_t;
+        item_slot[k % kItemSlots] = t;
+        mbar_arrive(bItemFull(k));           // publishes the slot (release)
+        if (t < 0) break;
+        next_t = claim_item(p, n_items);     // the atomic's latency overlaps this item's loads
         const Item it = decode_item(p, t);
         // the previous item's last QK^T has finished reading the Q buffer
         if (k > 0 && !(ok = ctl.wait(bQFree, (k - 1) & 1))) break;
@@ -552,8 +566,9 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       int c0 = 0;            // chunks of earlier items (global chunk index base)
       if (p.debug_never) ok = ctl.wait(bNever, 0);
       for (int k = 0; ok; ++k) {
-        const int t = item_at(k);
-        if (t >= n_items) break;
+        if (!(ok = ctl.wait(bItemFull(k), uint32_t(k / kItemSlots) & 1u))) break;
+        const int t = item_slot[k % kItemSlots];
+        if (t < 0) break;
         const Item it = decode_item(p, t);
         const int nch = it.len * CPB;
         if (!(ok = ctl.wait(bQFull, k & 1))) break;
@@ -638,8 +653,10 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     };
     if (p.debug_never) ok = __all_sync(0xffffffffu, ctl.wait(bNever, 0));
     for (int k = 0; ok; ++k) {
-      const int t = item_at(k);
-      if (t >= n_items) break;
+      ok = __all_sync(0xffffffffu, ctl.wait(bItemFull(k), uint32_t(k / kItemSlots) & 1u));
+      if (!ok) break;
+      const int t = item_slot[k % kItemSlots];
+      if (t < 0) break;
       const Item it = decode_item(p, t);
       const int nch = it.len * CPB;
       const int diag_first = it.diag_last ? nch - CPB : nch;   // first chunk of the diagonal block
@@ -911,6 +928,10 @@ int launch_instance(const ForwardArgs& a, dev::Params p) {
   } else {
     grid = 8;
   }
+  if (!a.debug_never) {
+    e = cudaMemsetAsync(p.work_counter, 0, sizeof(uint32_t), static_cast<cudaStream_t>(a.stream));
+    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing the work counter: ") + cudaGetErrorString(e));
+  }
   kern<<<grid, dev::kThreads, smem, static_cast<cudaStream_t>(a.stream)>>>(mq, mk, mv, mo, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
@@ -929,6 +950,7 @@ int launch_forward(const ForwardArgs& a) {
   p.order = L->d_order;
   p.lse = a.lse;
   p.status = L->d_status;
+  p.work_counter = L->d_status + kWorkCounterWord;
   p.n = a.n;
   p.nb = L->nb;
   p.heads = a.heads;
@@ -959,6 +981,7 @@ int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int3
   p.order = order;
   p.lse = a.lse;
   p.status = status;
+  p.work_counter = status + kWorkCounterWord;
   p.n = a.n;
   p.nb = L->nb;
   p.heads = a.heads;

@@ -35,6 +35,10 @@ int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out
 
 // Device status bits.
 constexpr uint32_t kStatusTimeout = 1u;
+// The 256-byte status block that follows a layout's arrays (and heads the
+// allocation-free scratch) holds the status word at word 0 and the kernel's
+// work counter at word 32, on its own 128-byte line.
+constexpr int kWorkCounterWord = 32;
 
 // Launch description handed to the kernel launcher (bsa_fwd_sm100a.cu).
 struct ForwardArgs {
