@@ -285,6 +285,35 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Two fp32 lanes at once (sm_100 packed FP32): each lane rounds exactly as
+// the scalar instruction would.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+__device__ __forceinline__ void mul2(float& d0, float& d1, float b) {
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %2};\n\t"
+      "mul.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(b));
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -339,8 +368,8 @@ struct KernelShape {
   static_assert(4 * (HD / 64) * kWarpStage == 2 * kTileBytes, "o staging fills two V slots");
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffPend = kOffMisc + 16;             // producer's pending-staging FIFO
-  static constexpr int kOffItems = kOffPend + 32;            // claimed item indices, ring of 8
-  static constexpr int kSmemUsed = kOffItems + 4 * kItemSlots;
+  static constexpr int kOffItems = kOffPend + 32;            // claimed, decoded items, ring of 8
+  static constexpr int kSmemUsed = kOffItems + 32 * kItemSlots;
   static constexpr int kColS = 0;                            // S buffers: columns 0..63, 64..127
   static constexpr int kColO = 2 * kChunk;
   static constexpr uint32_t kTmemCols = 256;
@@ -434,7 +463,19 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   const uint32_t bStageFree = bOFree + 24u;
   const uint32_t bItemFull0 = bOFree + 32u;
   auto bItemFull = [&](int k) { return bItemFull0 + 8u * (k % kItemSlots); };
-  volatile int* item_slot = reinterpret_cast<volatile int*>(gbase + S::kOffItems);
+  // slot k % 8: {valid, row, start, len, h0, kvh, diag_last}
+  volatile int* item_ring = reinterpret_cast<volatile int*>(gbase + S::kOffItems);
+  auto read_item = [&](int k, Item& it) -> bool {
+    volatile int* e = item_ring + 8 * (k % kItemSlots);
+    if (!e[0]) return false;
+    it.row = e[1];
+    it.start = e[2];
+    it.len = e[3];
+    it.h0 = e[4];
+    it.kvh = e[5];
+    it.diag_last = e[6] != 0;
+    return true;
+  };
   auto bKFull = [&](int c) { return bKFull0 + 8u * (c % kKSlots); };
   auto bVFull = [&](int c) { return bVFull0 + 8u * (c % kVSlots); };
   auto bSFull = [&](int c) { return bSFull0 + 8u * (c & 1); };
@@ -503,11 +544,19 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       int next_t = ok ? claim_item(p, n_items) : -1;
       for (int k = 0; ok; ++k) {
         const int t = next_t;
-        item_slot[k % kItemSlots] = t;
+        Item it{};
+        if (t >= 0) it = decode_item(p, t);
+        volatile int* e = item_ring + 8 * (k % kItemSlots);
+        e[0] = t >= 0;
+        e[1] = it.row;
+        e[2] = it.start;
+        e[3] = it.len;
+        e[4] = it.h0;
+        e[5] = it.kvh;
+        e[6] = it.diag_last;
         mbar_arrive(bItemFull(k));           // publishes the slot (release)
         if (t < 0) break;
         next_t = claim_item(p, n_items);     // the atomic's latency overlaps this item's loads
-        const Item it = decode_item(p, t);
         // the previous item's last QK^T has finished reading the Q buffer
         if (k > 0 && !(ok = ctl.wait(bQFree, (k - 1) & 1))) break;
         mbar_expect_tx(bQFull, S::kQBytes);
@@ -567,9 +616,8 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       if (p.debug_never) ok = ctl.wait(bNever, 0);
       for (int k = 0; ok; ++k) {
         if (!(ok = ctl.wait(bItemFull(k), uint32_t(k / kItemSlots) & 1u))) break;
-        const int t = item_slot[k % kItemSlots];
-        if (t < 0) break;
-        const Item it = decode_item(p, t);
+        Item it;
+        if (!read_item(k, it)) break;
         const int nch = it.len * CPB;
         if (!(ok = ctl.wait(bQFull, k & 1))) break;
         tc_fence_after();
@@ -655,9 +703,8 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     for (int k = 0; ok; ++k) {
       ok = __all_sync(0xffffffffu, ctl.wait(bItemFull(k), uint32_t(k / kItemSlots) & 1u));
       if (!ok) break;
-      const int t = item_slot[k % kItemSlots];
-      if (t < 0) break;
-      const Item it = decode_item(p, t);
+      Item it;
+      if (!read_item(k, it)) break;
       const int nch = it.len * CPB;
       const int diag_first = it.diag_last ? nch - CPB : nch;   // first chunk of the diagonal block
       if (nch == 0) release_stage();
@@ -670,44 +717,86 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         if (q == 0) release_stage();
         tc_fence_after();
         float sv[kChunk];
-        tmem_ld32(lane_base + S::kColS + s * kChunk, sv);
-        tmem_ld32(lane_base + S::kColS + s * kChunk + 32, sv + 32);
-        tmem_wait_ld();
-        if (q >= diag_first) {
-          // causal mask inside the diagonal block: key (chunk offset + c) > row
-          const int lim = rl - (q - diag_first) * kChunk;
+        const uint32_t s_col = lane_base + S::kColS + s * kChunk;
+        const bool masked = q >= diag_first;
+        // causal mask inside the diagonal block: key (chunk offset + c) > row
+        const int lim = rl - (q - diag_first) * kChunk;
+        auto load_s = [&]() {
+          tmem_ld32(s_col, sv);
+          tmem_ld32(s_col + 32, sv + 32);
+          tmem_wait_ld();
+          if (masked) {
 #pragma unroll
-          for (int c = 0; c < kChunk; ++c)
-            if (c > lim) sv[c] = -INFINITY;
-        }
-        float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+            for (int c = 0; c < kChunk; ++c)
+              if (c > lim) sv[c] = -INFINITY;
+          }
+        };
+        // P = exp2(S * scale * log2 e - m) in place, with four running sums
+        float s0, s1, s2, s3;
+        auto exp_pass = [&](float neg_m) {
+          s0 = s1 = s2 = s3 = 0.f;
 #pragma unroll
-        for (int c = 4; c < kChunk; c += 4) {
-          mx0 = fmaxf(mx0, sv[c]);
-          mx1 = fmaxf(mx1, sv[c + 1]);
-          mx2 = fmaxf(mx2, sv[c + 2]);
-          mx3 = fmaxf(mx3, sv[c + 3]);
+          for (int c = 0; c < kChunk; c += 4) {
+            float x0, x1, x2, x3;
+            fma2(x0, x1, sv[c], sv[c + 1], sl2, neg_m);
+            fma2(x2, x3, sv[c + 2], sv[c + 3], sl2, neg_m);
+            sv[c] = ex2(x0);
+            sv[c + 1] = ex2(x1);
+            sv[c + 2] = ex2(x2);
+            sv[c + 3] = ex2(x3);
+            add2(s0, s1, sv[c], sv[c + 1]);
+            add2(s2, s3, sv[c + 2], sv[c + 3]);
+          }
+        };
+        load_s();
+        float m_new = m2, alpha = 1.f;
+        bool need = false;
+        if (q == 0) {
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < kChunk; c += 4) {
+            mx0 = max3(mx0, sv[c], sv[c + 1]);
+            mx1 = max3(mx1, sv[c + 2], sv[c + 3]);
+          }
+          m_new = fmaxf(mx0, mx1) * sl2;
+          exp_pass((m_new == -INFINITY) ? 0.f : -m_new);
+        } else {
+          // The running max is finite after the first chunk (its key 0 is
+          // never masked).  Exponentiate with it while this chunk's max is
+          // reduced alongside; a row moves its max only when the chunk's max
+          // exceeds it by more than the threshold, and then this chunk is
+          // recomputed from S (still in TMEM) with the new max.
+          const float neg_m = -m2;
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+          s0 = s1 = s2 = s3 = 0.f;
+#pragma unroll
+          for (int c = 0; c < kChunk; c += 4) {
+            mx0 = max3(mx0, sv[c], sv[c + 1]);
+            mx1 = max3(mx1, sv[c + 2], sv[c + 3]);
+            float x0, x1, x2, x3;
+            fma2(x0, x1, sv[c], sv[c + 1], sl2, neg_m);
+            fma2(x2, x3, sv[c + 2], sv[c + 3], sl2, neg_m);
+            sv[c] = ex2(x0);
+            sv[c + 1] = ex2(x1);
+            sv[c + 2] = ex2(x2);
+            sv[c + 3] = ex2(x3);
+            add2(s0, s1, sv[c], sv[c + 1]);
+            add2(s2, s3, sv[c + 2], sv[c + 3]);
+          }
+          const float mb = fmaxf(mx0, mx1) * sl2;
+          // Each row moves its own max (so rows never influence each other's
+          // rounding); the warp recomputes and passes over O when any moved.
+          need = mb > m2 + kRescaleThreshold;
+          if (need) {
+            m_new = mb;
+            alpha = ex2(m2 - m_new);
+          }
+          if (__any_sync(0xffffffffu, need)) {
+            load_s();
+            exp_pass(-m_new);
+          }
         }
-        const float mb = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-        // Each row moves its own max (so rows never influence each other's
-        // rounding); the warp passes over O when any of its rows moved.
-        const bool need = q > 0 && mb > m2 + kRescaleThreshold;
-        const float m_new = (q == 0 || need) ? mb : m2;
-        const float alpha = need ? ex2(m2 - m_new) : 1.f;
         const bool resc = __any_sync(0xffffffffu, need);
-        const float neg_m = (m_new == -INFINITY) ? 0.f : -m_new;
-        float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-#pragma unroll
-        for (int c = 0; c < kChunk; c += 4) {
-          sv[c] = ex2(fmaf(sv[c], sl2, neg_m));
-          sv[c + 1] = ex2(fmaf(sv[c + 1], sl2, neg_m));
-          sv[c + 2] = ex2(fmaf(sv[c + 2], sl2, neg_m));
-          sv[c + 3] = ex2(fmaf(sv[c + 3], sl2, neg_m));
-          s0 += sv[c];
-          s1 += sv[c + 1];
-          s2 += sv[c + 2];
-          s3 += sv[c + 3];
-        }
         l = l * alpha + ((s0 + s1) + (s2 + s3));
         if (resc) {
           // O must hold PV_{sc-1} before it is rescaled; only rescaling chunks wait.
@@ -720,7 +809,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             tmem_ld32(lane_base + S::kColO + c * 32, ov);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+            for (int e = 0; e < 32; e += 2) mul2(ov[e], ov[e + 1], alpha);
             tmem_st32(lane_base + S::kColO + c * 32, ov);
           }
         }
