@@ -87,7 +87,7 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     const size_t b_ci = std::max<size_t>(1, lay->col_idx.size()) * sizeof(int32_t);
     const size_t b_or = lay->order.size() * sizeof(int32_t);
     const size_t o_ci = round_up(b_rp, 256), o_or = o_ci + round_up(b_ci, 256);
-    const size_t o_st = o_or + round_up(b_or, 256), total = o_st + 256;
+    const size_t o_st = o_or + round_up(b_or, 256), total = o_st + bsa::kStatusBlockBytes;
     void* base = nullptr;
     e = cudaMalloc(&base, total);
     if (e != cudaSuccess) {
@@ -103,7 +103,7 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
       e = cudaMemcpy(c + o_ci, lay->col_idx.data(), lay->col_idx.size() * sizeof(int32_t),
                      cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(c + o_or, lay->order.data(), b_or, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemset(c + o_st, 0, 256);
+    if (e == cudaSuccess) e = cudaMemset(c + o_st, 0, bsa::kStatusBlockBytes);
     if (e != cudaSuccess) {
       cudaFree(base);
       delete lay;

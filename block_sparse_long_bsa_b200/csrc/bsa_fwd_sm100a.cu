@@ -1039,7 +1039,10 @@ int launch_forward(const ForwardArgs& a) {
   p.order = L->d_order;
   p.lse = a.lse;
   p.status = L->d_status;
-  p.work_counter = L->d_status + kWorkCounterWord;
+  {
+    const uint32_t call = const_cast<bsa_layout*>(L)->calls.fetch_add(1, std::memory_order_relaxed);
+    p.work_counter = L->d_status + 64 + size_t(call % kWorkCounters) * 32;
+  }
   p.n = a.n;
   p.nb = L->nb;
   p.heads = a.heads;
@@ -1070,7 +1073,7 @@ int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int3
   p.order = order;
   p.lse = a.lse;
   p.status = status;
-  p.work_counter = status + kWorkCounterWord;
+  p.work_counter = status + kScratchCounterWord;
   p.n = a.n;
   p.nb = L->nb;
   p.heads = a.heads;

@@ -2,6 +2,7 @@
 // sm_100a kernel launcher.  Not part of the public interface.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <string>
 #include <vector>
@@ -23,6 +24,7 @@ struct bsa_layout {
   const int32_t* d_col_idx = nullptr;
   const int32_t* d_order = nullptr;
   uint32_t* d_status = nullptr;   // bit 0: a device wait ran out
+  std::atomic<uint32_t> calls{0};  // forwards launched (picks each call's work counter)
 };
 
 namespace bsa {
@@ -35,10 +37,14 @@ int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out
 
 // Device status bits.
 constexpr uint32_t kStatusTimeout = 1u;
-// The 256-byte status block that follows a layout's arrays (and heads the
-// allocation-free scratch) holds the status word at word 0 and the kernel's
-// work counter at word 32, on its own 128-byte line.
-constexpr int kWorkCounterWord = 32;
+// The status block that follows a layout's arrays holds the status word at
+// word 0 and, from byte 256 on, kWorkCounters work counters, one per 128-byte
+// line: forward number c of a layout uses counter c % kWorkCounters, so up to
+// that many forwards on one layout may be in flight at once.  The
+// allocation-free scratch has one counter, at word 32.
+constexpr int kWorkCounters = 64;
+constexpr size_t kStatusBlockBytes = 256 + size_t(kWorkCounters) * 128;
+constexpr int kScratchCounterWord = 32;
 
 // Launch description handed to the kernel launcher (bsa_fwd_sm100a.cu).
 struct ForwardArgs {

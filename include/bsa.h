@@ -127,12 +127,12 @@ int bsa_layout_order(const bsa_layout* layout, const int32_t** order, int* count
  * device; B in {64, 128}; d in {64, 128}; heads and kv_heads >= 1,
  * heads % kv_heads == 0, heads % layout_heads == 0; scale finite and > 0;
  * q, k, v, o non-null and 16-byte aligned; lse non-null and 4-byte aligned.
- * o and lse must not overlap the inputs.  Enqueues a 4-byte clear of the
- * layout's work counter and one kernel; returns after enqueueing them.  The
- * work counter lives in the layout's device block, so two forwards with the
- * same layout must not run at the same time on different streams (calls on
- * one stream are ordered and fine).  A device-side wait that runs out (never
- * expected) makes the kernel return early and is reported by bsa_get_status. */
+ * o and lse must not overlap the inputs.  Enqueues a 4-byte clear of a work
+ * counter and one kernel; returns after enqueueing them.  Each call takes the
+ * next of 64 work counters held in the layout's device block, so forwards
+ * with the same layout may run at the same time on different streams (up to
+ * 64 in flight at once).  A device-side wait that runs out (never expected)
+ * makes the kernel return early and is reported by bsa_get_status. */
 int bsa_forward(const void* q, const void* k, const void* v,
                 const bsa_layout* layout, int B, int n, int heads, int kv_heads,
                 int d, float scale, void* o, float* lse, void* stream);

@@ -227,6 +227,28 @@ def test_run_to_run_bitwise_deterministic():
     lay.close()
 
 
+def test_concurrent_forwards_on_one_layout():
+    # Forwards sharing a layout on different streams, overlapping on the GPU,
+    # each claim their own work counter: every result equals the serial one.
+    n, B, d = 8192, 64, 128
+    dev = torch.cuda.current_device()
+    lay = bsa.Layout(OL.DYADIC, n, B, 1, dev, window=2, global_first=1, dyadic_kmin=2)
+    _, (q, k, v) = device_inputs(8, 4, n, d)
+    o_ref, l_ref = bsa.attention(q, k, v, lay)
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in range(4)]
+    outs = []
+    for rep in range(3):
+        for s in streams:
+            with torch.cuda.stream(s):
+                outs.append(bsa.attention(q, k, v, lay, stream=s))
+    torch.cuda.synchronize()
+    for o, l in outs:
+        assert torch.equal(o, o_ref) and torch.equal(l, l_ref)
+    bsa.bsa_get_status(lay.handle)
+    lay.close()
+
+
 # ----------------------------------------------------------------- boundary
 def test_invalid_arguments_launch_nothing():
     n, B, d = 1024, 64, 128
