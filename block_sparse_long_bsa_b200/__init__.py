@@ -32,8 +32,8 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "B
                 7: "BSA_ERR_DEVICE_TIMEOUT"}
 
 EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_order", "bsa_forward",
-            "bsa_forward_noalloc", "bsa_get_status", "bsa_debug_timeout_probe", "bsa_free",
-            "bsa_last_error"]
+            "bsa_forward_noalloc", "bsa_decode", "bsa_get_status", "bsa_debug_timeout_probe",
+            "bsa_free", "bsa_last_error"]
 
 
 class BsaError(RuntimeError):
@@ -77,6 +77,8 @@ def load_library(path: str = LIB_PATH):
         lib.bsa_forward.restype = I
         lib.bsa_forward_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P]
         lib.bsa_forward_noalloc.restype = I
+        lib.bsa_decode.argtypes = [P, P, P, P, I, I, P, P, I, I, I, I, F, P, P, P]
+        lib.bsa_decode.restype = I
         lib.bsa_get_status.argtypes = [P, P]
         lib.bsa_get_status.restype = I
         lib.bsa_debug_timeout_probe.argtypes = [P, I, U64, P]
@@ -174,6 +176,40 @@ def bsa_forward_noalloc(q, k, v, layout: int, B: int, n: int, heads: int, kv_hea
     lib = load_library()
     _check(lib.bsa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), layout, B, n, heads, kv_heads, d,
                                    ctypes.c_float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_decode(q, k_cache, v_cache, page_table, max_blocks: int, num_pages: int, positions,
+               layout: int, batch: int, heads: int, kv_heads: int, d: int, scale: float,
+               o, lse, stream=None) -> None:
+    """Enqueue one selected-page decode step (see include/bsa.h)."""
+    lib = load_library()
+    _check(lib.bsa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table), max_blocks,
+                          num_pages, _ptr(positions), layout, batch, heads, kv_heads, d,
+                          ctypes.c_float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def decode(q, k_cache, v_cache, page_table, positions, layout: "Layout", batch: int,
+           scale: float | None = None, o=None, lse=None, stream=None):
+    """torch convenience: q [batch*H, d]; caches [pages, H_kv, B, d] bf16;
+    page_table [batch, max_blocks] and positions [batch] int32, all on the GPU."""
+    import torch
+    heads, d = q.shape
+    kv_heads = k_cache.shape[1] * batch
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((heads,), dtype=torch.float32, device=q.device)
+    for t in (q, k_cache, v_cache, o):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise BsaError(1, "q, caches and o must be contiguous bf16 tensors")
+    for t in (page_table, positions):
+        if t.dtype != torch.int32 or not t.is_contiguous():
+            raise BsaError(1, "page_table and positions must be contiguous int32 tensors")
+    bsa_decode(q, k_cache, v_cache, page_table, page_table.shape[1], k_cache.shape[0], positions,
+               layout.handle, batch, heads, kv_heads, d, scale, o, lse, stream)
+    return o, lse
 
 
 def bsa_get_status(layout: int, stream=None) -> None:

@@ -200,6 +200,8 @@ int bsa_get_status(const bsa_layout* layout, void* stream) {
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("status read: ") + cudaGetErrorString(e));
   if (word & bsa::kStatusTimeout)
     return set_error(BSA_ERR_DEVICE_TIMEOUT, "a device-side wait ran out; the kernel returned early");
+  if (word & bsa::kStatusBadIndex)
+    return set_error(BSA_ERR_SHAPE, "a decode position or page number was out of range; its row got o = 0");
   return BSA_OK;
 }
 

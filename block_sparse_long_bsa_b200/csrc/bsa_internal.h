@@ -37,6 +37,7 @@ int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out
 
 // Device status bits.
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBadIndex = 2u;   // a decode position or page number was out of range
 // The status block that follows a layout's arrays holds the status word at
 // word 0 and, from byte 256 on, kWorkCounters work counters, one per 128-byte
 // line: forward number c of a layout uses counter c % kWorkCounters, so up to

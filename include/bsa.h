@@ -173,6 +173,39 @@ int bsa_forward_noalloc(const void* q, const void* k, const void* v,
                         const bsa_layout* layout, int B, int n, int heads, int kv_heads,
                         int d, float scale, void* o, float* lse, void* stream);
 
+/* Selected-page decode ("BF1: A Causal Dyadic Sparse-Attention Retrofit for
+ * Efficient Long-Context Transformers", section 5: one new query token per
+ * sequence reads the same block route as prefill, over a cache of keys and
+ * values; the route is planned once, in the layout, and reused every step).
+ * For sequence b (0 <= b < batch) whose new token is at position
+ * t = positions[b] (block i = t / B, B the layout's block size), query row
+ * f = b*H + h (H = heads / batch) attends to the cached keys u <= t of the key
+ * blocks that block row i of layout head f % layout_heads keeps, reading
+ * key/value head h / (H / Hkv) of the sequence (Hkv = kv_heads / batch):
+ *   s_u = scale * <q[f], k_u>,  lse[f] = ln sum_u exp(s_u),
+ *   o[f] = sum_u exp(s_u - lse[f]) v_u;
+ * a row with no allowed key gets o = 0 and lse = -inf.  Layouts (device
+ * memory, caller-owned): q, o [heads][d] bf16; k_cache, v_cache
+ * [num_pages][Hkv][B][d] bf16, page p holding the B consecutive tokens of one
+ * logical block for every key/value head of a sequence (rows past a
+ * sequence's end are never read); page_table [batch][max_blocks] int32, the
+ * page of logical block j of sequence b; positions [batch] int32; lse [heads]
+ * fp32.  The new token's own key and value must already be in the cache.
+ * Requirements (checked before launch; errors launch nothing): layout on the
+ * current device; B in {64, 128}; d in {64, 128}; batch, heads, kv_heads >= 1;
+ * heads and kv_heads multiples of batch; H a multiple of Hkv and of
+ * layout_heads; max_blocks >= the layout's blocks; num_pages >= 1; scale
+ * finite and > 0; pointers non-null, q, caches and o 16-byte aligned, the rest
+ * 4-byte aligned.  A position outside [0, n) or a page outside
+ * [0, num_pages) read on the device is not dereferenced: that row gets o = 0,
+ * lse = -inf and bsa_get_status then reports BSA_ERR_SHAPE.  Launches one
+ * kernel and returns after enqueueing it; no allocation, no synchronisation. */
+int bsa_decode(const void* q, const void* k_cache, const void* v_cache,
+               const int32_t* page_table, int max_blocks, int num_pages,
+               const int32_t* positions, const bsa_layout* layout, int batch,
+               int heads, int kv_heads, int d, float scale, void* o, float* lse,
+               void* stream);
+
 /* Release a layout and its device arrays (NULL is a no-op).  The caller must
  * make sure no forward that uses it is still running. */
 void bsa_free(bsa_layout* layout);
