@@ -462,6 +462,7 @@ def main():
             if name == w.name:
                 continue
             per_config[name] = bench_other(WORKLOADS[name], dev, stream, flush, bsa, torch)
+    decode = bench_decode(dev, stream, flush, bsa, torch) if rank == 0 and not args.no_per_config else None
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -505,6 +506,7 @@ def main():
             "roofline": roofline,
             "cpu_baseline": cpu,
             "per_config": per_config,
+            "decode": decode,
         }
         print(json.dumps(line), flush=True)
     sampler.stop()
@@ -545,6 +547,60 @@ def bench_other(w, dev, stream, flush, bsa, torch, steps=10, warmup=3):
     return {"ms_median": med, "tflops": flops / (med * 1e-3) / 1e12, "kept_pairs": pairs,
             "hbm_gbs_compulsory": compulsory / (med * 1e-3) / 1e9,
             "data": "torch.randn on device, seed 1234"}
+
+
+def bench_decode(dev, stream, flush, bsa, torch, batches=(1, 32), steps=20, warmup=3):
+    """Selected-page decode on the headline route: each sequence's new token at
+    the last position of a 32K context, reading its block row's kept pages
+    through a shuffled page table.  Reports time per step and the unique
+    key/value bytes of the kept pages (what a step must read) per second."""
+    w = WORKLOADS[HEADLINE]
+    lay = bsa.Layout.for_workload(w, dev)
+    row_ptr, col_idx = lay.csr()
+    H, hkv, B, d, n = w.q_heads, w.kv_heads_per_seq, w.B, w.d, w.n
+    nb = -(-n // B)
+    t = n - 1
+    i = t // B
+    kept = [int(j) for j in col_idx[row_ptr[i]:row_ptr[i + 1]]]
+    toks = sum(min(B, t + 1 - j * B) for j in kept)
+    hbm = float(load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    out = {"workload": f"BF1 dyadic route, token at position {t} of a {n}-token context, "
+                       f"{H}/{hkv} heads, d={d}, B={B} pages",
+           "kept_blocks": len(kept), "l2": "256 MiB written between steps"}
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(99)
+    for batch in batches:
+        pages = batch * nb
+        kc = torch.randn((pages, hkv, B, d), device=dev, generator=gen).to(torch.bfloat16)
+        vc = torch.randn((pages, hkv, B, d), device=dev, generator=gen).to(torch.bfloat16)
+        table = torch.randperm(pages, device=dev, generator=gen).to(torch.int32).view(batch, nb).contiguous()
+        q = torch.randn((batch * H, d), device=dev, generator=gen).to(torch.bfloat16)
+        pos = torch.full((batch,), t, dtype=torch.int32, device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((batch * H,), dtype=torch.float32, device=dev)
+        ev = []
+        for st in range(warmup + steps):
+            flush.fill_(float(st))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            bsa.bsa_decode(q, kc, vc, table, nb, pages, pos, lay.handle, batch, batch * H,
+                           batch * hkv, d, 1.0 / math.sqrt(d), o, lse, stream)
+            b.record(stream)
+            if st >= warmup:
+                ev.append((a, b))
+        torch.cuda.synchronize()
+        bsa.bsa_get_status(lay.handle)
+        ts = sorted(a.elapsed_time(b) for a, b in ev)
+        us = ts[len(ts) // 2] * 1e3
+        kv_bytes = batch * hkv * toks * d * 2 * 2
+        io_bytes = batch * H * d * 2 * 2 + batch * H * 4
+        gbs = (kv_bytes + io_bytes) / (us * 1e-6) / 1e9
+        out[f"batch_{batch}"] = {"us_per_step": us, "tokens_per_s": batch / (us * 1e-6),
+                                 "bytes_per_step": kv_bytes + io_bytes, "gbs": gbs,
+                                 "frac_of_measured_hbm": gbs / hbm}
+        del kc, vc, table, q, pos, o, lse
+    lay.close()
+    return out
 
 
 if __name__ == "__main__":

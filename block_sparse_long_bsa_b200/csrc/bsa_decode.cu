@@ -7,22 +7,27 @@
 //
 // A query row is a single vector, so the step is a stream over the kept
 // pages' keys and values (HBM/L2 bound, no matrix product to hand to the
-// tensor cores).  One CTA per query row; its 8 warps take the kept blocks in
-// turn.  For each block a warp scores its keys (lane l owns keys l, l + 32,
-// ..., reading each key row in 16-byte pieces against q held in shared
-// memory), folds them into its running max and sum, and accumulates
-// P V with lanes across d (each key row read as one coalesced line).  The
-// warps' partial (max, sum, o) are then merged in shared memory.  Everything is
-// fp32 (P is not rounded to bf16); o is stored as bf16 and lse in fp32.
+// tensor cores).  One CTA serves two query rows of a key/value head's group
+// when they share a route (one layout head, an even group), else one row, so
+// a group's rows read each kept page once.  Its 16 warps take the kept blocks in turn.  For a
+// block, 8 lanes cooperate on each key row (16-byte loads, the row read as
+// one coalesced line; a 3-step shuffle tree sums the dot product), four rows
+// per step, scoring the row against all G queries held in shared memory; the
+// scores go through shared memory for the block's max, exponentials and sum
+// (an fp32 online softmax per query), and P V is accumulated with lanes across
+// d.  The warps' partial (max, sum, o) are then merged in shared memory.
+// Everything is fp32 (P is not rounded to bf16); o is stored as bf16 and lse
+// in fp32.
 //
 // Positions and page numbers come from device memory: a position outside
 // [0, n) or a page outside [0, num_pages) is not read; the kernel records a
 // status bit (reported by bsa_get_status) and writes o = 0, lse = -inf for
-// that row.
+// the rows of that CTA.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <mutex>
 #include <string>
 
 #include "bsa_internal.h"
@@ -30,7 +35,8 @@
 namespace bsa {
 namespace dec {
 
-constexpr int kWarps = 8;
+constexpr int kTileBudget = 192 * 1024;   // shared memory for the warps' K/V tiles
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a copy that takes longer than 1 s is abandoned
 constexpr float kLn2 = 0.693147180559945309f;
 
 struct DecodeParams {
@@ -49,39 +55,95 @@ struct DecodeParams {
   float scale_log2;
 };
 
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// One contiguous tile global -> shared by the bulk-copy engine (no multicast),
+// completing the given mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+// Bounded wait for a phase of an mbarrier; false if it did not complete in time.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = gtimer();
+  while (true) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}\n"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    if (ok) return true;
+    if (gtimer() - t0 > kWaitLimitNs) return false;
+  }
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
+// G query rows per CTA (2 when the rows of a group share a route, else 1).
 template <int BLK, int HD>
-__global__ void __launch_bounds__(kWarps * 32) bsa_decode_kernel(const DecodeParams p) {
-  constexpr int KPL = BLK / 32;       // keys per lane in a block
+__host__ __device__ constexpr int warps_for() {   // as many warps as K and V tiles of a page fit the budget, at most 6
+  return kTileBudget / (2 * BLK * HD * 2) < 6 ? kTileBudget / (2 * BLK * HD * 2) : 6;
+}
+
+template <int BLK, int HD, int G>
+__global__ void __launch_bounds__(warps_for<BLK, HD>() * 32) bsa_decode_kernel(const DecodeParams p) {
+  constexpr int kWarps = warps_for<BLK, HD>();
+  constexpr int CPL = HD / 8;         // key columns per lane (8 lanes per key row)
   constexpr int DPL = HD / 32;        // o columns per lane
-  __shared__ float sq[HD];
-  __shared__ float sm[kWarps], sl[kWarps];
-  __shared__ float so[kWarps][HD];
+  constexpr uint32_t kTile = BLK * HD * 2;   // one page's K (or V) tile of one head
+  extern __shared__ __align__(128) uint8_t dyn[];   // per warp: K tile, V tile
+  __shared__ __align__(8) uint64_t tile_bar[kWarps];
+  __shared__ float sq[G][HD];
+  __shared__ float sp[kWarps][G][BLK];          // scores, then P, of a warp's block
+  __shared__ float sm[kWarps][G], sl[kWarps][G];
+  __shared__ float so[kWarps][G][HD];
   __shared__ int s_bad;
-  const int f = blockIdx.x;
-  const int b = f / p.H, h = f - b * p.H;
-  const int hk = h / p.g;
+  // the CTA's rows f0 .. f0 + G - 1 (G divides g, so they share a key/value head)
+  const int f0 = blockIdx.x * G;
+  const int b = f0 / p.H;
+  const int hk = (f0 - b * p.H) / p.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float sl2 = p.scale_log2;
-  for (int c = threadIdx.x; c < HD; c += blockDim.x) sq[c] = __bfloat162float(p.q[size_t(f) * HD + c]);
+  for (int c = threadIdx.x; c < G * HD; c += blockDim.x)
+    sq[c / HD][c % HD] = __bfloat162float(p.q[size_t(f0) * HD + c]);
   if (threadIdx.x == 0) s_bad = 0;
+  if (lane == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&tile_bar[warp])) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   __syncthreads();
+  const uint32_t bar = smem_u32(&tile_bar[warp]);
+  const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(dyn + size_t(warp) * 2 * kTile);
+  const __nv_bfloat16* vt = kt + BLK * HD;
+  int loads = 0;                      // tiles pairs this warp has brought in (barrier phases)
 
   const int t = p.positions[b];
   const bool pos_ok = t >= 0 && t < p.n;
-  float m = -INFINITY, l = 0.f;       // this warp's running max (exp2 units) and sum
-  float acc[DPL];
+  float m[G], l[G], acc[G][DPL];
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  for (int gq = 0; gq < G; ++gq) {
+    m[gq] = -INFINITY;
+    l[gq] = 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[gq][e] = 0.f;
+  }
   if (pos_ok) {
     const int i = t / BLK;
-    const size_t row = size_t(f % p.L) * p.nb + i;
+    const size_t row = size_t(f0 % p.L) * p.nb + i;
     const int start = p.row_ptr[row], len = p.row_ptr[row + 1] - start;
+    const int sub = lane >> 3, part = lane & 7;   // key row within a step of 4, column slice
     for (int e = warp; e < len; e += kWarps) {
       const int j = p.col_idx[start + e];
       const int page = p.page_table[size_t(b) * p.max_blocks + j];
@@ -90,110 +152,182 @@ __global__ void __launch_bounds__(kWarps * 32) bsa_decode_kernel(const DecodePar
         continue;
       }
       const size_t tile = (size_t(page) * p.hkv + hk) * BLK * HD;
-      const __nv_bfloat16* kt = p.kc + tile;
-      const __nv_bfloat16* vt = p.vc + tile;
-      // scores of this lane's keys
-      float s[KPL];
-      float bm = -INFINITY;
+      // this block's K and V tiles into the warp's buffers, one bulk copy each
+      __syncwarp();                      // every lane is done with the previous tiles
+      if (lane == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads before the copy
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTile)
+                     : "memory");
+        bulk_load(smem_u32(kt), p.kc + tile, kTile, bar);
+        bulk_load(smem_u32(vt), p.vc + tile, kTile, bar);
+      }
+      const bool landed = bar_wait(bar, uint32_t(loads) & 1u);
+      ++loads;
+      if (!__all_sync(0xffffffffu, landed)) {
+        if (lane == 0) s_bad = 2;
+        break;
+      }
+      // ---- scores: rows 4 * step + sub, columns part * CPL ..
+#pragma unroll 4
+      for (int step = 0; step < BLK / 4; ++step) {
+        const int r = step * 4 + sub;
+        const uint4* kr = reinterpret_cast<const uint4*>(kt + size_t(r) * HD + part * CPL);
+        float dot[G];
 #pragma unroll
-      for (int kk = 0; kk < KPL; ++kk) {
-        const int r = lane + 32 * kk;
-        const uint4* kr = reinterpret_cast<const uint4*>(kt + size_t(r) * HD);
-        float dot = 0.f;
+        for (int gq = 0; gq < G; ++gq) dot[gq] = 0.f;
 #pragma unroll
-        for (int c8 = 0; c8 < HD / 8; ++c8) {
-          const uint4 w = __ldg(kr + c8);
+        for (int c8 = 0; c8 < CPL / 8; ++c8) {
+          const uint4 w = kr[c8];
           const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&w);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 kv = __bfloat1622float2(pr[e]);
-            dot = fmaf(kv.x, sq[c8 * 8 + 2 * e], dot);
-            dot = fmaf(kv.y, sq[c8 * 8 + 2 * e + 1], dot);
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 kv = __bfloat1622float2(pr[e2]);
+            const int c = part * CPL + c8 * 8 + 2 * e2;
+#pragma unroll
+            for (int gq = 0; gq < G; ++gq) {
+              dot[gq] = fmaf(kv.x, sq[gq][c], dot[gq]);
+              dot[gq] = fmaf(kv.y, sq[gq][c + 1], dot[gq]);
+            }
           }
         }
-        const bool allowed = j * BLK + r <= t;   // causal; other blocks of the route are earlier
-        s[kk] = allowed ? dot * sl2 : -INFINITY;
-        bm = fmaxf(bm, s[kk]);
+#pragma unroll
+        for (int gq = 0; gq < G; ++gq) {
+          dot[gq] += __shfl_xor_sync(0xffffffffu, dot[gq], 1);
+          dot[gq] += __shfl_xor_sync(0xffffffffu, dot[gq], 2);
+          dot[gq] += __shfl_xor_sync(0xffffffffu, dot[gq], 4);
+        }
+        if (part == 0) {
+          const bool allowed = j * BLK + r <= t;   // causal; other blocks of the route are earlier
+#pragma unroll
+          for (int gq = 0; gq < G; ++gq) sp[warp][gq][r] = allowed ? dot[gq] * sl2 : -INFINITY;
+        }
       }
+      __syncwarp();
+      // ---- online softmax per query over this block's keys
+      float alpha[G];
+      bool any = false;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-      if (bm == -INFINITY) continue;             // nothing allowed in this block
-      const float m_new = fmaxf(m, bm);
-      const float alpha = ex2(m - m_new);        // 0 when m = -inf
-      float psum = 0.f;
+      for (int gq = 0; gq < G; ++gq) {
+        float bm = -INFINITY;
 #pragma unroll
-      for (int kk = 0; kk < KPL; ++kk) {
-        s[kk] = ex2(s[kk] - m_new);
-        psum += s[kk];
+        for (int r = lane; r < BLK; r += 32) bm = fmaxf(bm, sp[warp][gq][r]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+        const float m_new = fmaxf(m[gq], bm);
+        alpha[gq] = (m_new == -INFINITY) ? 1.f : ex2(m[gq] - m_new);   // 0 when m was -inf
+        float psum = 0.f;
+#pragma unroll
+        for (int r = lane; r < BLK; r += 32) {
+          const float pv = (m_new == -INFINITY) ? 0.f : ex2(sp[warp][gq][r] - m_new);
+          sp[warp][gq][r] = pv;
+          psum += pv;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+        l[gq] = l[gq] * alpha[gq] + psum;
+        m[gq] = m_new;
+        any = any || bm != -INFINITY;
       }
+      __syncwarp();
+      if (!any) continue;                        // nothing allowed in this block
+      // ---- O += P V: lane owns columns lane * DPL ..
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
-      l = l * alpha + psum;
-      m = m_new;
+      for (int gq = 0; gq < G; ++gq)
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] *= alpha;
-      // O += P V: lane owns columns lane * DPL ..
-#pragma unroll
-      for (int kk = 0; kk < KPL; ++kk) {
+        for (int e2 = 0; e2 < DPL; ++e2) acc[gq][e2] *= alpha[gq];
 #pragma unroll 8
-        for (int src = 0; src < 32; ++src) {
-          const float pu = __shfl_sync(0xffffffffu, s[kk], src);
-          const __nv_bfloat16* vr = vt + size_t(src + 32 * kk) * HD + lane * DPL;
-          if constexpr (DPL == 4) {
-            const uint2 w = __ldg(reinterpret_cast<const uint2*>(vr));
-            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
-            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
-            acc[0] = fmaf(pu, a.x, acc[0]);
-            acc[1] = fmaf(pu, a.y, acc[1]);
-            acc[2] = fmaf(pu, c.x, acc[2]);
-            acc[3] = fmaf(pu, c.y, acc[3]);
-          } else {
-            const uint32_t w = __ldg(reinterpret_cast<const unsigned int*>(vr));
-            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
-            acc[0] = fmaf(pu, a.x, acc[0]);
-            acc[1] = fmaf(pu, a.y, acc[1]);
-          }
+      for (int r = 0; r < BLK; ++r) {
+        const __nv_bfloat16* vr = vt + size_t(r) * HD + lane * DPL;
+        float vv[DPL];
+        if constexpr (DPL == 4) {
+          const uint2 w = *reinterpret_cast<const uint2*>(vr);
+          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
+          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
+          vv[0] = a.x;
+          vv[1] = a.y;
+          vv[2] = c.x;
+          vv[3] = c.y;
+        } else {
+          const uint32_t w = *reinterpret_cast<const unsigned int*>(vr);
+          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
+          vv[0] = a.x;
+          vv[1] = a.y;
+        }
+#pragma unroll
+        for (int gq = 0; gq < G; ++gq) {
+          const float pu = sp[warp][gq][r];
+#pragma unroll
+          for (int e2 = 0; e2 < DPL; ++e2) acc[gq][e2] = fmaf(pu, vv[e2], acc[gq][e2]);
         }
       }
+      __syncwarp();
     }
   } else if (threadIdx.x == 0) {
     s_bad = 1;
   }
   // merge the warps' partial softmax states
-  if (lane == 0) {
-    sm[warp] = m;
-    sl[warp] = l;
-  }
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) so[warp][lane * DPL + e] = acc[e];
+  for (int gq = 0; gq < G; ++gq) {
+    if (lane == 0) {
+      sm[warp][gq] = m[gq];
+      sl[warp][gq] = l[gq];
+    }
+#pragma unroll
+    for (int e2 = 0; e2 < DPL; ++e2) so[warp][gq][lane * DPL + e2] = acc[gq][e2];
+  }
   __syncthreads();
-  float M = -INFINITY;
+  // a refused index (or a copy that never landed): the CTA's rows are o = 0,
+  // lse = -inf.  Leave no copy in flight into shared memory.
+  if (lane == 0 && loads > 0) bar_wait(bar, uint32_t(loads - 1) & 1u);
+  __syncwarp();
+  const bool bad = s_bad != 0;
+  for (int c = threadIdx.x; c < G * HD; c += blockDim.x) {
+    const int gq = c / HD, col = c % HD;
+    float M = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm[w]);
-  float Lsum = 0.f;
-  float wgt[kWarps];
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm[w][gq]);
+    float Lsum = 0.f, v = 0.f;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    wgt[w] = (M == -INFINITY) ? 0.f : ex2(sm[w] - M);
-    Lsum += wgt[w] * sl[w];
+    for (int w = 0; w < kWarps; ++w) {
+      const float wt = (M == -INFINITY) ? 0.f : ex2(sm[w][gq] - M);
+      Lsum += wt * sl[w][gq];
+      v += wt * so[w][gq][col];
+    }
+    const bool ok = Lsum > 0.f && !bad;
+    p.o[size_t(f0 + gq) * HD + col] = __float2bfloat16_rn(ok ? v / Lsum : 0.f);
+    if (col == 0) p.lse[f0 + gq] = ok ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
   }
-  const bool bad = s_bad != 0;           // a refused index: the whole row is o = 0, lse = -inf
-  const float inv = (Lsum > 0.f && !bad) ? 1.f / Lsum : 0.f;
-  for (int c = threadIdx.x; c < HD; c += blockDim.x) {
-    float v = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) v += wgt[w] * so[w][c];
-    p.o[size_t(f) * HD + c] = __float2bfloat16_rn(v * inv);
+  if (threadIdx.x == 0 && bad) atomicOr(p.status, s_bad == 2 ? kStatusTimeout : kStatusBadIndex);
+}
+
+template <int BLK, int HD, int G>
+int launch_g(const DecodeParams& p, int heads, cudaStream_t s) {
+  auto kern = bsa_decode_kernel<BLK, HD, G>;
+  constexpr int kWarps = warps_for<BLK, HD>();
+  const int smem = kWarps * 2 * BLK * HD * 2;
+  // the attribute is a property of the function: set it once per device
+  static std::mutex mu;
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) return set_error(BSA_ERR_CUDA, "cannot query the device");
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done[dev]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode smem: ") + cudaGetErrorString(e));
+      done[dev] = true;
+    }
   }
-  if (threadIdx.x == 0) {
-    p.lse[f] = (Lsum > 0.f && !bad) ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
-    if (bad) atomicOr(p.status, kStatusBadIndex);
-  }
+  kern<<<heads / G, kWarps * 32, smem, s>>>(p);
+  return BSA_OK;
 }
 
 template <int BLK, int HD>
 int launch(const DecodeParams& p, int heads, cudaStream_t s) {
-  bsa_decode_kernel<BLK, HD><<<heads, kWarps * 32, 0, s>>>(p);
+  // two query rows of a key/value head's group per CTA when they share a route
+  const int st = (p.L == 1 && p.g % 2 == 0) ? launch_g<BLK, HD, 2>(p, heads, s) : launch_g<BLK, HD, 1>(p, heads, s);
+  if (st != BSA_OK) return st;
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
   return BSA_OK;

@@ -995,12 +995,24 @@ int launch_instance(const ForwardArgs& a, dev::Params p) {
   int smem = S::kSmemUsed;
   const int floor_bytes = (228 * 1024) / (MIN_CTAS + 1) + 1024;
   if (smem < floor_bytes) smem = floor_bytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+  // The shared-memory attribute belongs to the function and the SM count to
+  // the device: both are set / queried once per device.
+  static std::mutex mu;
+  static int sm_count[64] = {};
   int dev_id = 0, sms = 0;
-  e = cudaGetDevice(&dev_id);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
-  if (e != cudaSuccess || sms < 1) return set_error(BSA_ERR_CUDA, "cannot query the SM count");
+  cudaError_t e = cudaGetDevice(&dev_id);
+  if (e != cudaSuccess || dev_id < 0 || dev_id >= 64) return set_error(BSA_ERR_CUDA, "cannot query the device");
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (sm_count[dev_id] == 0) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev_id);
+      if (e != cudaSuccess || sms < 1) return set_error(BSA_ERR_CUDA, "cannot query the SM count");
+      sm_count[dev_id] = sms;
+    }
+    sms = sm_count[dev_id];
+  }
   CUtensorMap mq, mk, mv, mo;
   std::memset(&mo, 0, sizeof(mo));
   std::memset(&mq, 0, sizeof(mq));

@@ -196,10 +196,11 @@ int bsa_forward_noalloc(const void* q, const void* k, const void* v,
  * heads and kv_heads multiples of batch; H a multiple of Hkv and of
  * layout_heads; max_blocks >= the layout's blocks; num_pages >= 1; scale
  * finite and > 0; pointers non-null, q, caches and o 16-byte aligned, the rest
- * 4-byte aligned.  A position outside [0, n) or a page outside
- * [0, num_pages) read on the device is not dereferenced: that row gets o = 0,
- * lse = -inf and bsa_get_status then reports BSA_ERR_SHAPE.  Launches one
- * kernel and returns after enqueueing it; no allocation, no synchronisation. */
+ * 4-byte aligned; num_pages must be the number of pages the caches hold.  A
+ * position outside [0, n) or a page outside [0, num_pages) read on the device
+ * is not dereferenced: the rows it concerns get o = 0, lse = -inf and
+ * bsa_get_status then reports BSA_ERR_SHAPE.  Launches one kernel and returns
+ * after enqueueing it; no allocation, no synchronisation. */
 int bsa_decode(const void* q, const void* k_cache, const void* v_cache,
                const int32_t* page_table, int max_blocks, int num_pages,
                const int32_t* positions, const bsa_layout* layout, int batch,
