@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "B
                 4: "BSA_ERR_NONCAUSAL", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_OOM",
                 7: "BSA_ERR_DEVICE_TIMEOUT"}
 
-EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_order", "bsa_forward",
+EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_csc", "bsa_layout_order", "bsa_forward",
             "bsa_forward_noalloc", "bsa_decode", "bsa_get_status", "bsa_debug_timeout_probe",
             "bsa_free", "bsa_last_error"]
 
@@ -70,6 +70,10 @@ def load_library(path: str = LIB_PATH):
                                        ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
                                        ctypes.POINTER(I), ctypes.POINTER(I)]
         lib.bsa_layout_csr.restype = I
+        lib.bsa_layout_csc.argtypes = [P, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                       ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                       ctypes.POINTER(I), ctypes.POINTER(I)]
+        lib.bsa_layout_csc.restype = I
         lib.bsa_layout_order.argtypes = [P, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
                                          ctypes.POINTER(I)]
         lib.bsa_layout_order.restype = I
@@ -137,6 +141,20 @@ def bsa_build_layout(kind: int, n: int, B: int, layout_heads: int = 1, device: i
     out = ctypes.c_void_p()
     _check(lib.bsa_build_layout(ctypes.byref(spec), n, B, layout_heads, device, ctypes.byref(out)))
     return out.value
+
+
+def bsa_layout_csc(layout: int):
+    """Copies of the transposed layout (col_ptr, row_idx) as int32 numpy arrays."""
+    lib = load_library()
+    cp = ctypes.POINTER(ctypes.c_int32)()
+    ri = ctypes.POINTER(ctypes.c_int32)()
+    cols, nnz = ctypes.c_int(), ctypes.c_int()
+    _check(lib.bsa_layout_csc(layout, ctypes.byref(cp), ctypes.byref(ri), ctypes.byref(cols),
+                              ctypes.byref(nnz)))
+    col_ptr = np.ctypeslib.as_array(cp, shape=(cols.value + 1,)).copy()
+    row_idx = (np.ctypeslib.as_array(ri, shape=(nnz.value,)).copy() if nnz.value
+               else np.zeros(0, np.int32))
+    return col_ptr, row_idx
 
 
 def bsa_layout_csr(layout: int):

@@ -87,7 +87,10 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     const size_t b_ci = std::max<size_t>(1, lay->col_idx.size()) * sizeof(int32_t);
     const size_t b_or = lay->order.size() * sizeof(int32_t);
     const size_t o_ci = round_up(b_rp, 256), o_or = o_ci + round_up(b_ci, 256);
-    const size_t o_st = o_or + round_up(b_or, 256), total = o_st + bsa::kStatusBlockBytes;
+    const size_t b_cp = lay->col_ptr.size() * sizeof(int32_t);
+    const size_t b_ri = std::max<size_t>(1, lay->row_idx.size()) * sizeof(int32_t);
+    const size_t o_cp = o_or + round_up(b_or, 256), o_ri = o_cp + round_up(b_cp, 256);
+    const size_t o_st = o_ri + round_up(b_ri, 256), total = o_st + bsa::kStatusBlockBytes;
     void* base = nullptr;
     e = cudaMalloc(&base, total);
     if (e != cudaSuccess) {
@@ -103,6 +106,10 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
       e = cudaMemcpy(c + o_ci, lay->col_idx.data(), lay->col_idx.size() * sizeof(int32_t),
                      cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(c + o_or, lay->order.data(), b_or, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(c + o_cp, lay->col_ptr.data(), b_cp, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !lay->row_idx.empty())
+      e = cudaMemcpy(c + o_ri, lay->row_idx.data(), lay->row_idx.size() * sizeof(int32_t),
+                     cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(c + o_st, 0, bsa::kStatusBlockBytes);
     if (e != cudaSuccess) {
       cudaFree(base);
@@ -114,6 +121,8 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     lay->d_row_ptr = reinterpret_cast<const int32_t*>(c);
     lay->d_col_idx = reinterpret_cast<const int32_t*>(c + o_ci);
     lay->d_order = reinterpret_cast<const int32_t*>(c + o_or);
+    lay->d_col_ptr = reinterpret_cast<const int32_t*>(c + o_cp);
+    lay->d_row_idx = reinterpret_cast<const int32_t*>(c + o_ri);
     lay->d_status = reinterpret_cast<uint32_t*>(c + o_st);
     lay->device = device;
     if (prev >= 0 && prev != device) cudaSetDevice(prev);
@@ -136,6 +145,16 @@ int bsa_layout_order(const bsa_layout* layout, const int32_t** order, int* count
   if (!layout) return set_error(BSA_ERR_INVALID_ARG, "layout is NULL");
   if (order) *order = layout->order.data();
   if (count) *count = int(layout->order.size());
+  return BSA_OK;
+}
+
+int bsa_layout_csc(const bsa_layout* layout, const int32_t** col_ptr, const int32_t** row_idx,
+                   int* cols, int* nnz) {
+  if (!layout) return set_error(BSA_ERR_INVALID_ARG, "layout is NULL");
+  if (col_ptr) *col_ptr = layout->col_ptr.data();
+  if (row_idx) *row_idx = layout->row_idx.data();
+  if (cols) *cols = int(layout->col_ptr.size()) - 1;
+  if (nnz) *nnz = int(layout->row_idx.size());
   return BSA_OK;
 }
 

@@ -19,10 +19,14 @@ struct bsa_layout {
   std::vector<int32_t> row_ptr;   // [L*nb + 1]
   std::vector<int32_t> col_idx;   // [nnz]
   std::vector<int32_t> order;     // [L*nb], longest row first per layout head
+  std::vector<int32_t> col_ptr;   // [L*nb + 1]: transposed layout (CSC), per layout head
+  std::vector<int32_t> row_idx;   // [nnz]: query blocks keeping each key block, ascending
   void* d_base = nullptr;         // single device allocation holding the arrays below
   const int32_t* d_row_ptr = nullptr;
   const int32_t* d_col_idx = nullptr;
   const int32_t* d_order = nullptr;
+  const int32_t* d_col_ptr = nullptr;
+  const int32_t* d_row_idx = nullptr;
   uint32_t* d_status = nullptr;   // bit 0: a device wait ran out
   std::atomic<uint32_t> calls{0};  // forwards launched (picks each call's work counter)
 };

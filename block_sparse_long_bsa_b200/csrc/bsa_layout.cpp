@@ -140,6 +140,27 @@ int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out
     }
   }
 
+  // The transposed layout (for gradients of keys and values): for layout head
+  // h and key block j, the query blocks whose rows keep j, ascending.
+  out->col_ptr.assign(size_t(L) * nb + 1, 0);
+  out->row_idx.assign(out->col_idx.size(), 0);
+  for (int h = 0; h < L; ++h)
+    for (int i = 0; i < nb; ++i) {
+      const size_t r = size_t(h) * nb + i;
+      for (int32_t e = out->row_ptr[r]; e < out->row_ptr[r + 1]; ++e)
+        ++out->col_ptr[size_t(h) * nb + out->col_idx[e] + 1];
+    }
+  for (size_t c = 0; c + 1 < out->col_ptr.size(); ++c) out->col_ptr[c + 1] += out->col_ptr[c];
+  {
+    std::vector<int32_t> fill(out->col_ptr.begin(), out->col_ptr.end() - 1);
+    for (int h = 0; h < L; ++h)
+      for (int i = 0; i < nb; ++i) {
+        const size_t r = size_t(h) * nb + i;
+        for (int32_t e = out->row_ptr[r]; e < out->row_ptr[r + 1]; ++e)
+          out->row_idx[fill[size_t(h) * nb + out->col_idx[e]]++] = i;
+      }
+  }
+
   // Longest row first within each layout head; equal lengths keep block order.
   out->order.resize(size_t(L) * nb);
   for (int h = 0; h < L; ++h) {

@@ -115,6 +115,13 @@ int bsa_layout_csr(const bsa_layout* layout, const int32_t** row_ptr,
  * query block processed at rank r for layout head h.  count = layout_heads*nb. */
 int bsa_layout_order(const bsa_layout* layout, const int32_t** order, int* count);
 
+/* Read-only host view of the transposed layout: for layout head h and key
+ * block j, row_idx[col_ptr[h*nb + j] .. col_ptr[h*nb + j + 1]) lists, in
+ * ascending order, the query blocks whose rows keep j (the key/value side of
+ * the gradients reads the layout this way).  cols = layout_heads * nb. */
+int bsa_layout_csc(const bsa_layout* layout, const int32_t** col_ptr,
+                   const int32_t** row_idx, int* cols, int* nnz);
+
 /* Block-sparse causal attention forward on the caller's stream.
  * For every folded query head f and token t (block i = t / B):
  *   s_tu = scale * <q[f][t], k[g][u]>,  g = f / (heads / kv_heads),

@@ -143,6 +143,19 @@ def to_csr(sets: list):
     return row_ptr, col_idx
 
 
+def to_csc(sets: list):
+    """The transposed layout over columns (h, j) in order h-major: for each key
+    block j of layout head h, the query blocks i whose kept set holds j, in
+    ascending order.  (col_ptr, row_idx) lists."""
+    col_ptr, row_idx = [0], []
+    for per_head in sets:
+        nb = len(per_head)
+        for j in range(nb):
+            row_idx.extend(i for i in range(nb) if j in per_head[i])
+            col_ptr.append(len(row_idx))
+    return col_ptr, row_idx
+
+
 def block_mask(sets_one_head: list):
     """Dense n_b x n_b 0/1 block mask M_B of one layout head."""
     nb = len(sets_one_head)

@@ -92,6 +92,12 @@ def _check_order(rp, order, L, nb):
 def test_layout_edge_cases_bit_exact(lib, kind, n, B, L, kw):
     rp, ci, order = _csr_from_lib(kind, n, B, L, **kw)
     sets = OL.kept_sets(kind, n, B, L, **kw)
+    lay = bsa.Layout(kind, n, B, L, -1, **kw)
+    cp, ri = bsa.bsa_layout_csc(lay.handle)
+    lay.close()
+    ocp, ori = OL.to_csc(sets)
+    np.testing.assert_array_equal(cp, np.array(ocp, dtype=np.int32))
+    np.testing.assert_array_equal(ri, np.array(ori, dtype=np.int32))
     orp, oci = OL.to_csr(sets)
     np.testing.assert_array_equal(rp, np.array(orp, dtype=np.int32))
     np.testing.assert_array_equal(ci, np.array(oci, dtype=np.int32))
