@@ -1,4 +1,5 @@
-"""Python binding of ``libbsa.so``: block-sparse causal attention forward on B200.
+"""Python binding of ``libbsa.so``: block-sparse causal attention on B200
+(forward, gradients, selected-page decode).
 
 Argument marshalling only.  Every step of the computation runs in the
 library's CUDA kernel or its host layout compiler; this module converts Python
@@ -7,9 +8,11 @@ non-zero status codes into :class:`BsaError`.  There is no fallback: if the
 shared library is missing or cannot be loaded, every call raises.
 
 Names follow the C ABI: ``bsa_build_layout``, ``bsa_layout_csr``,
-``bsa_layout_order``, ``bsa_forward``, ``bsa_get_status``,
-``bsa_debug_timeout_probe``, ``bsa_free`` and ``bsa_last_error``; the
-``Layout`` class and ``attention`` are conveniences over them.
+``bsa_layout_csc``, ``bsa_layout_order``, ``bsa_layout_segments``,
+``bsa_forward``, ``bsa_forward_noalloc``, ``bsa_backward``, ``bsa_decode``,
+``bsa_get_status``, ``bsa_debug_timeout_probe``, ``bsa_free`` and
+``bsa_last_error``; the ``Layout`` class, ``attention``, ``attention_backward``
+and ``decode`` are conveniences over them.
 """
 from __future__ import annotations
 
@@ -31,9 +34,9 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "B
                 4: "BSA_ERR_NONCAUSAL", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_OOM",
                 7: "BSA_ERR_DEVICE_TIMEOUT"}
 
-EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_csc", "bsa_layout_order", "bsa_forward",
-            "bsa_forward_noalloc", "bsa_decode", "bsa_get_status", "bsa_debug_timeout_probe",
-            "bsa_free", "bsa_last_error"]
+EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_csc", "bsa_layout_order",
+            "bsa_layout_segments", "bsa_forward", "bsa_forward_noalloc", "bsa_backward", "bsa_decode",
+            "bsa_get_status", "bsa_debug_timeout_probe", "bsa_free", "bsa_last_error"]
 
 
 class BsaError(RuntimeError):
@@ -83,6 +86,12 @@ def load_library(path: str = LIB_PATH):
         lib.bsa_forward_noalloc.restype = I
         lib.bsa_decode.argtypes = [P, P, P, P, I, I, P, P, I, I, I, I, F, P, P, P]
         lib.bsa_decode.restype = I
+        lib.bsa_backward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, P, P, P]
+        lib.bsa_backward.restype = I
+        lib.bsa_layout_segments.argtypes = [P, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                            ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                            ctypes.POINTER(I), ctypes.POINTER(I)]
+        lib.bsa_layout_segments.restype = I
         lib.bsa_get_status.argtypes = [P, P]
         lib.bsa_get_status.restype = I
         lib.bsa_debug_timeout_probe.argtypes = [P, I, U64, P]
@@ -157,6 +166,20 @@ def bsa_layout_csc(layout: int):
     return col_ptr, row_idx
 
 
+def bsa_layout_segments(layout: int):
+    """Copies of the key/value-gradient work list: (seg_ptr [L+1], segs [count, 3])."""
+    lib = load_library()
+    sp = ctypes.POINTER(ctypes.c_int32)()
+    sg = ctypes.POINTER(ctypes.c_int32)()
+    lh, cnt = ctypes.c_int(), ctypes.c_int()
+    _check(lib.bsa_layout_segments(layout, ctypes.byref(sp), ctypes.byref(sg), ctypes.byref(lh),
+                                   ctypes.byref(cnt)))
+    seg_ptr = np.ctypeslib.as_array(sp, shape=(lh.value + 1,)).copy()
+    segs = (np.ctypeslib.as_array(sg, shape=(cnt.value * 3,)).copy().reshape(-1, 3) if cnt.value
+            else np.zeros((0, 3), np.int32))
+    return seg_ptr, segs
+
+
 def bsa_layout_csr(layout: int):
     """Copies of (row_ptr, col_idx) as int32 numpy arrays."""
     lib = load_library()
@@ -204,6 +227,43 @@ def bsa_decode(q, k_cache, v_cache, page_table, max_blocks: int, num_pages: int,
     _check(lib.bsa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table), max_blocks,
                           num_pages, _ptr(positions), layout, batch, heads, kv_heads, d,
                           ctypes.c_float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_backward(q, k, v, o, lse, dout, layout: int, B: int, n: int, heads: int, kv_heads: int,
+                 d: int, scale: float, dq, dk, dv, workspace, stream=None) -> None:
+    """Enqueue the gradients of the forward (see include/bsa.h)."""
+    lib = load_library()
+    _check(lib.bsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), layout, B, n,
+                            heads, kv_heads, d, ctypes.c_float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                            _ptr(workspace), _stream(stream)))
+
+
+def attention_backward(q, k, v, o, lse, dout, layout: "Layout", scale: float | None = None,
+                       dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """torch convenience: the forward's tensors plus dout [heads, n, d] bf16;
+    returns fp32 (dq, dk, dv), allocating what is not given."""
+    import torch
+    heads, n, d = q.shape
+    kv_heads = k.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    for t in (q, k, v, o, dout):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise BsaError(1, "q, k, v, o and dout must be contiguous bf16 tensors")
+    if dq is None:
+        dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.empty(k.shape, dtype=torch.float32, device=q.device)
+    if dv is None:
+        dv = torch.empty(v.shape, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty((heads, n), dtype=torch.float32, device=q.device)
+    for t in (lse, dq, dk, dv, workspace):
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise BsaError(1, "lse, dq, dk, dv and workspace must be contiguous float32 tensors")
+    bsa_backward(q, k, v, o, lse, dout, layout.handle, layout.B, n, heads, kv_heads, d, scale,
+                 dq, dk, dv, workspace, stream)
+    return dq, dk, dv
 
 
 def decode(q, k_cache, v_cache, page_table, positions, layout: "Layout", batch: int,

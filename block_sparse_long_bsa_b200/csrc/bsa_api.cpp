@@ -90,7 +90,10 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     const size_t b_cp = lay->col_ptr.size() * sizeof(int32_t);
     const size_t b_ri = std::max<size_t>(1, lay->row_idx.size()) * sizeof(int32_t);
     const size_t o_cp = o_or + round_up(b_or, 256), o_ri = o_cp + round_up(b_cp, 256);
-    const size_t o_st = o_ri + round_up(b_ri, 256), total = o_st + bsa::kStatusBlockBytes;
+    const size_t b_sp = lay->seg_ptr.size() * sizeof(int32_t);
+    const size_t b_sg = std::max<size_t>(1, lay->segs.size()) * sizeof(int32_t);
+    const size_t o_sp = o_ri + round_up(b_ri, 256), o_sg = o_sp + round_up(b_sp, 256);
+    const size_t o_st = o_sg + round_up(b_sg, 256), total = o_st + bsa::kStatusBlockBytes;
     void* base = nullptr;
     e = cudaMalloc(&base, total);
     if (e != cudaSuccess) {
@@ -110,6 +113,9 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     if (e == cudaSuccess && !lay->row_idx.empty())
       e = cudaMemcpy(c + o_ri, lay->row_idx.data(), lay->row_idx.size() * sizeof(int32_t),
                      cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(c + o_sp, lay->seg_ptr.data(), b_sp, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !lay->segs.empty())
+      e = cudaMemcpy(c + o_sg, lay->segs.data(), lay->segs.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(c + o_st, 0, bsa::kStatusBlockBytes);
     if (e != cudaSuccess) {
       cudaFree(base);
@@ -123,6 +129,8 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     lay->d_order = reinterpret_cast<const int32_t*>(c + o_or);
     lay->d_col_ptr = reinterpret_cast<const int32_t*>(c + o_cp);
     lay->d_row_idx = reinterpret_cast<const int32_t*>(c + o_ri);
+    lay->d_seg_ptr = reinterpret_cast<const int32_t*>(c + o_sp);
+    lay->d_segs = reinterpret_cast<const int32_t*>(c + o_sg);
     lay->d_status = reinterpret_cast<uint32_t*>(c + o_st);
     lay->device = device;
     if (prev >= 0 && prev != device) cudaSetDevice(prev);
@@ -168,6 +176,16 @@ static int check_device(const bsa_layout* layout) {
   if (cur != layout->device)
     return set_error(BSA_ERR_INVALID_ARG, "layout lives on device " + std::to_string(layout->device) +
                                               " but the current device is " + std::to_string(cur));
+  return BSA_OK;
+}
+
+int bsa_layout_segments(const bsa_layout* layout, const int32_t** seg_ptr, const int32_t** segs,
+                        int* layout_heads, int* count) {
+  if (!layout) return set_error(BSA_ERR_INVALID_ARG, "layout is NULL");
+  if (seg_ptr) *seg_ptr = layout->seg_ptr.data();
+  if (segs) *segs = layout->segs.data();
+  if (layout_heads) *layout_heads = layout->L;
+  if (count) *count = int(layout->segs.size() / 3);
   return BSA_OK;
 }
 

@@ -21,12 +21,17 @@ struct bsa_layout {
   std::vector<int32_t> order;     // [L*nb], longest row first per layout head
   std::vector<int32_t> col_ptr;   // [L*nb + 1]: transposed layout (CSC), per layout head
   std::vector<int32_t> row_idx;   // [nnz]: query blocks keeping each key block, ascending
+  std::vector<int32_t> seg_ptr;   // [L + 1]: column segments of layout head h are seg_ptr[h] .. seg_ptr[h+1]
+  std::vector<int32_t> segs;      // [3 * segments]: (key block j, first row_idx entry, entries <= kColumnSegment)
+  int max_segs = 0;               // most segments of one layout head
   void* d_base = nullptr;         // single device allocation holding the arrays below
   const int32_t* d_row_ptr = nullptr;
   const int32_t* d_col_idx = nullptr;
   const int32_t* d_order = nullptr;
   const int32_t* d_col_ptr = nullptr;
   const int32_t* d_row_idx = nullptr;
+  const int32_t* d_seg_ptr = nullptr;
+  const int32_t* d_segs = nullptr;
   uint32_t* d_status = nullptr;   // bit 0: a device wait ran out
   std::atomic<uint32_t> calls{0};  // forwards launched (picks each call's work counter)
 };
@@ -38,6 +43,10 @@ int set_error(int status, const std::string& msg);
 
 // Host layout compiler (bsa_layout.cpp).  Fills row_ptr/col_idx/order/max_row.
 int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out);
+
+// Longest run of query blocks one key/value-gradient work item takes from a
+// column of the transposed layout.
+constexpr int kColumnSegment = 16;
 
 // Device status bits.
 constexpr uint32_t kStatusTimeout = 1u;

@@ -161,6 +161,36 @@ int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out
       }
   }
 
+  // Column segments (the work list of the key/value gradients): each column
+  // cut into runs of at most kColumnSegment query blocks, so a key block read
+  // by every query block (a global first block) is shared out like any other;
+  // per layout head, longest segment first, equal lengths in column order.
+  out->seg_ptr.assign(size_t(L) + 1, 0);
+  out->segs.clear();
+  for (int h = 0; h < L; ++h) {
+    const size_t first = out->segs.size() / 3;
+    for (int j = 0; j < nb; ++j) {
+      const int32_t c0 = out->col_ptr[size_t(h) * nb + j], c1 = out->col_ptr[size_t(h) * nb + j + 1];
+      for (int32_t e = c0; e < c1; e += kColumnSegment) {
+        out->segs.push_back(j);
+        out->segs.push_back(e);
+        out->segs.push_back(std::min<int32_t>(kColumnSegment, c1 - e));
+      }
+    }
+    const size_t count = out->segs.size() / 3 - first;
+    std::vector<int32_t> idx(count);
+    std::iota(idx.begin(), idx.end(), 0);
+    const int32_t* sg = out->segs.data() + first * 3;
+    std::stable_sort(idx.begin(), idx.end(), [sg](int32_t a, int32_t b) { return sg[3 * a + 2] > sg[3 * b + 2]; });
+    std::vector<int32_t> sorted(count * 3);
+    for (size_t x = 0; x < count; ++x)
+      for (int w = 0; w < 3; ++w) sorted[3 * x + w] = sg[3 * idx[x] + w];
+    std::copy(sorted.begin(), sorted.end(), out->segs.begin() + first * 3);
+    if (out->segs.size() / 3 > size_t(INT32_MAX)) return set_error(BSA_ERR_SHAPE, "too many column segments");
+    out->seg_ptr[h + 1] = int32_t(out->segs.size() / 3);
+    out->max_segs = std::max<int>(out->max_segs, int(count));
+  }
+
   // Longest row first within each layout head; equal lengths keep block order.
   out->order.resize(size_t(L) * nb);
   for (int h = 0; h < L; ++h) {

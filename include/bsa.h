@@ -1,5 +1,6 @@
 /*
- * bsa.h -- C ABI of the B200 (sm_100a) block-sparse causal attention forward.
+ * bsa.h -- C ABI of the B200 (sm_100a) block-sparse causal attention
+ * forward, its gradients and selected-page decode.
  *
  * What the library computes ("Block-Sparse Attention", ai-model-reference,
  * sections "How It Works" and "Math Or Compute Schema"): the sequence of n
@@ -213,6 +214,38 @@ int bsa_decode(const void* q, const void* k_cache, const void* v_cache,
                const int32_t* positions, const bsa_layout* layout, int batch,
                int heads, int kv_heads, int d, float scale, void* o, float* lse,
                void* stream);
+
+/* Gradients of the forward ("BF1: A Causal Dyadic Sparse-Attention Retrofit
+ * for Efficient Long-Context Transformers", section 4: the operator is gated
+ * on its gradients and adaptation trains through the route).  Given the
+ * forward's inputs, its outputs o and lse, and dout = dL/do, for the same
+ * allowed pairs (t, u) and P_tu = exp(s_tu - lse_t):
+ *   D_t = <dout_t, o_t>,  dS_tu = P_tu (<dout_t, v_u> - D_t),
+ *   dq_t = scale sum_u dS_tu k_u,  dk_u = scale sum_t dS_tu q_t,
+ *   dv_u = sum_t P_tu dout_t,
+ * dk and dv summing over the query heads of the key/value head's group.
+ * Layouts: q, o, dout [heads][n][d] bf16; k, v [kv_heads][n][d] bf16; lse
+ * [heads][n] fp32 (the forward's, natural log); dq [heads][n][d] fp32; dk,
+ * dv [kv_heads][n][d] fp32; workspace [heads][n] fp32 (receives D).  All
+ * device memory, caller-owned, not overlapping.  Requirements as for
+ * bsa_forward (checked before launch; errors launch nothing), plus dout, dq,
+ * dk, dv 16-byte aligned and workspace 4-byte aligned.  Enqueues two clears
+ * (dk, dv) and three kernels (D, dq, dk/dv) on the stream and returns; the
+ * dk/dv kernel adds its partial sums in fp32, so their summation order (and
+ * last bits) may differ from run to run.  A wait that runs out is reported
+ * by bsa_get_status as for the forward. */
+int bsa_backward(const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dout, const bsa_layout* layout,
+                 int B, int n, int heads, int kv_heads, int d, float scale,
+                 float* dq, float* dk, float* dv, float* workspace, void* stream);
+
+/* Read-only host view of the key/value-gradient work list: for layout head
+ * h, segments seg_ptr[h] .. seg_ptr[h+1] - 1, segment s being the triple
+ * segs[3s .. 3s+2] = (key block j, first index into the transposed layout's
+ * row_idx, entry count <= 16), longest first.  Every column of the
+ * transposed layout is cut into runs of at most 16 query blocks. */
+int bsa_layout_segments(const bsa_layout* layout, const int32_t** seg_ptr,
+                        const int32_t** segs, int* layout_heads, int* count);
 
 /* Release a layout and its device arrays (NULL is a no-op).  The caller must
  * make sure no forward that uses it is still running. */

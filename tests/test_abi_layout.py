@@ -104,6 +104,46 @@ def test_layout_edge_cases_bit_exact(lib, kind, n, B, L, kw):
     _check_order(rp, order, L, OL.n_blocks(n, B))
 
 
+def _segments_from_csc(col_ptr, L, nb, seg=16):
+    """Columns cut into runs of at most `seg` entries, per layout head, stably
+    sorted by run length (longest first)."""
+    seg_ptr, out = [0], []
+    for h in range(L):
+        runs = []
+        for j in range(nb):
+            c0, c1 = col_ptr[h * nb + j], col_ptr[h * nb + j + 1]
+            for e in range(c0, c1, seg):
+                runs.append((j, e, min(seg, c1 - e)))
+        runs.sort(key=lambda r: -r[2])          # Python's sort is stable
+        out.extend(runs)
+        seg_ptr.append(len(out))
+    return np.array(seg_ptr, dtype=np.int32), np.array(out, dtype=np.int32).reshape(-1, 3)
+
+
+@pytest.mark.parametrize("kind,n,B,L,kw", [
+    (OL.DYADIC, 32768, 64, 1, dict(window=2, global_first=1, dyadic_kmin=2)),
+    (OL.BAND_GLOBAL, 32768, 128, 1, dict(window=2, global_first=1)),
+    (OL.RANDOM, 128 * 300, 128, 3, dict(density=0.3, seed=7)),
+    (OL.BAND_GLOBAL, 1, 64, 1, dict(window=3, global_first=1)),
+    (OL.RANDOM, 64 * 50, 64, 2, dict(density=0.0, seed=1)),
+])
+def test_gradient_work_segments_bit_exact(lib, kind, n, B, L, kw):
+    sets = OL.kept_sets(kind, n, B, L, **kw)
+    ocp, ori = OL.to_csc(sets)
+    want_ptr, want = _segments_from_csc(ocp, L, OL.n_blocks(n, B))
+    lay = bsa.Layout(kind, n, B, L, -1, **kw)
+    seg_ptr, segs = bsa.bsa_layout_segments(lay.handle)
+    lay.close()
+    np.testing.assert_array_equal(seg_ptr, want_ptr)
+    np.testing.assert_array_equal(segs, want)
+    # every (column, query block) entry is covered exactly once
+    covered = np.zeros(len(ori), dtype=np.int64)
+    for j, e, c in segs:
+        assert 1 <= c <= 16
+        covered[e:e + c] += 1
+    assert np.all(covered == 1)
+
+
 def test_explicit_mask_bit_exact_and_noncausal(lib):
     nb, B = 20, 64
     rng = np.random.default_rng(0)
