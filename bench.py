@@ -463,6 +463,9 @@ def main():
                 continue
             per_config[name] = bench_other(WORKLOADS[name], dev, stream, flush, bsa, torch)
     decode = bench_decode(dev, stream, flush, bsa, torch) if rank == 0 and not args.no_per_config else None
+    backward = ({name: bench_backward(WORKLOADS[name], dev, stream, flush, bsa, torch)
+                 for name in (HEADLINE, "band_global_32k")}
+                if rank == 0 and not args.no_per_config else None)
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -507,6 +510,7 @@ def main():
             "cpu_baseline": cpu,
             "per_config": per_config,
             "decode": decode,
+            "backward": backward,
         }
         print(json.dumps(line), flush=True)
     sampler.stop()
@@ -547,6 +551,53 @@ def bench_other(w, dev, stream, flush, bsa, torch, steps=10, warmup=3):
     return {"ms_median": med, "tflops": flops / (med * 1e-3) / 1e12, "kept_pairs": pairs,
             "hbm_gbs_compulsory": compulsory / (med * 1e-3) / 1e9,
             "data": "torch.randn on device, seed 1234"}
+
+
+def bench_backward(w, dev, stream, flush, bsa, torch, steps=10, warmup=3):
+    """Gradients (dq, dk, dv) of the forward on a workload: one bsa_backward
+    call per step (the D kernel, the dq kernel, the dk/dv kernel and two
+    clears), timed with CUDA events on the launching stream.  Effective
+    TFLOP/s counts 10 d flops per kept pair (the S, dP, dq, dk and dv
+    products, 2 d each); the kernels compute S and dP twice, 14 d per pair."""
+    lay = bsa.Layout.for_workload(w, dev)
+    row_ptr, col_idx = lay.csr()
+    pairs, flops_fwd, _ = workload_work(w, row_ptr, col_idx)
+    flops = flops_fwd * 10 // 4
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321)
+    q = torch.randn((w.heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    k = torch.randn((w.kv_heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    v = torch.randn((w.kv_heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    do = torch.randn((w.heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.heads, w.n), dtype=torch.float32, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    ws = torch.empty((w.heads, w.n), dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(w.d)
+    bsa.bsa_forward(q, k, v, lay.handle, w.B, w.n, w.heads, w.kv_heads, w.d, scale, o, lse, stream)
+    ev = []
+    for st in range(warmup + steps):
+        flush.fill_(float(st))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        bsa.bsa_backward(q, k, v, o, lse, do, lay.handle, w.B, w.n, w.heads, w.kv_heads, w.d, scale,
+                         dq, dk, dv, ws, stream)
+        b.record(stream)
+        if st >= warmup:
+            ev.append((a, b))
+    torch.cuda.synchronize()
+    bsa.bsa_get_status(lay.handle)
+    ts = sorted(a.elapsed_time(b) for a, b in ev)
+    med = ts[len(ts) // 2]
+    peak = float(load_peaks()[0].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    lay.close()
+    del q, k, v, do, o, lse, dq, dk, dv, ws
+    tf = flops / (med * 1e-3) / 1e12
+    return {"ms_median": med, "effective_tflops": tf, "frac_of_measured_peak": tf / peak,
+            "algorithmic_flops": flops, "kept_pairs": pairs, "launches_per_call": 3,
+            "data": "torch.randn on device, seed 4321; L2 flushed between steps"}
 
 
 def bench_decode(dev, stream, flush, bsa, torch, batches=(1, 32), steps=20, warmup=3):
