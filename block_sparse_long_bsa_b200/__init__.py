@@ -36,7 +36,8 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "B
 
 EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_csc", "bsa_layout_order",
             "bsa_layout_segments", "bsa_forward", "bsa_forward_noalloc", "bsa_backward", "bsa_decode",
-            "bsa_get_status", "bsa_debug_timeout_probe", "bsa_free", "bsa_last_error"]
+            "bsa_bsbr_workspace_bytes", "bsa_bsbr_retrieval", "bsa_get_status", "bsa_debug_timeout_probe",
+            "bsa_free", "bsa_last_error"]
 
 
 class BsaError(RuntimeError):
@@ -92,6 +93,10 @@ def load_library(path: str = LIB_PATH):
                                             ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
                                             ctypes.POINTER(I), ctypes.POINTER(I)]
         lib.bsa_layout_segments.restype = I
+        lib.bsa_bsbr_workspace_bytes.argtypes = [I, I, I, I]
+        lib.bsa_bsbr_workspace_bytes.restype = ctypes.c_size_t
+        lib.bsa_bsbr_retrieval.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, ctypes.c_size_t, P]
+        lib.bsa_bsbr_retrieval.restype = I
         lib.bsa_get_status.argtypes = [P, P]
         lib.bsa_get_status.restype = I
         lib.bsa_debug_timeout_probe.argtypes = [P, I, U64, P]
@@ -264,6 +269,36 @@ def attention_backward(q, k, v, o, lse, dout, layout: "Layout", scale: float | N
     bsa_backward(q, k, v, o, lse, dout, layout.handle, layout.B, n, heads, kv_heads, d, scale,
                  dq, dk, dv, workspace, stream)
     return dq, dk, dv
+
+
+def bsa_bsbr_workspace_bytes(n: int, B: int, kv_heads: int, d: int) -> int:
+    return int(load_library().bsa_bsbr_workspace_bytes(n, B, kv_heads, d))
+
+
+def bsa_bsbr_retrieval(q, k, v, layout: int, B: int, n: int, heads: int, kv_heads: int, d: int,
+                       scale: float, o, workspace, workspace_bytes: int, stream=None) -> None:
+    """Enqueue BSBR's between-chunk retrieval term, added to ``o`` (see include/bsa.h)."""
+    lib = load_library()
+    _check(lib.bsa_bsbr_retrieval(_ptr(q), _ptr(k), _ptr(v), layout, B, n, heads, kv_heads, d,
+                                  ctypes.c_float(scale), _ptr(o), _ptr(workspace), workspace_bytes,
+                                  _stream(stream)))
+
+
+def bsbr_attention(q, k, v, layout: "Layout", scale: float | None = None, workspace=None, stream=None):
+    """torch convenience: the whole BSBR attention output for a block-diagonal
+    ``layout`` (within-chunk forward, then the retrieval term added in place)."""
+    import torch
+    heads, n, d = q.shape
+    kv_heads = k.shape[0]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o, lse = attention(q, k, v, layout, scale=scale, stream=stream)
+    need = bsa_bsbr_workspace_bytes(n, layout.B, kv_heads, d)
+    if workspace is None:
+        workspace = torch.empty((max(need, 16) + 15) // 16 * 4, dtype=torch.float32, device=q.device)
+    bsa_bsbr_retrieval(q, k, v, layout.handle, layout.B, n, heads, kv_heads, d, scale, o, workspace,
+                       workspace.numel() * workspace.element_size(), stream)
+    return o, lse
 
 
 def decode(q, k_cache, v_cache, page_table, positions, layout: "Layout", batch: int,

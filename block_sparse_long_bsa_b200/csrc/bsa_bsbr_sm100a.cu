@@ -1,0 +1,724 @@
+// BSBR's between-chunk retrieval term for B200 (sm_100a) ("bsbr",
+// jvboid.dev/projects/bsbr, section "Solution"): each chunk of B tokens is
+// compressed into the state F_c = K_c^T V_c; chunk c retrieves from the
+// states of the chunks before it with softmax weights of its meta query
+// against their meta keys (R_c, H_c: means of q and k over a chunk), and its
+// tokens read the retrieved d x d state with their queries.  The result is
+// added to the within-chunk attention output (the block-diagonal layout of
+// the forward) already in o.
+//
+// Two launches: the state kernel (one CTA per key/value head and chunk:
+// F_c by one tcgen05 product, H_c by column sums) and the retrieval kernel
+// (one CTA per query head and chunk >= 1: meta weights, the weighted sum of
+// earlier states in fp32, and o += Q_c S_c by tcgen05 products with S split
+// into bf16 hi + lo parts).  The work is small and bound by memory traffic
+// and latency; the products go to the tensor cores so no fp32 ALU loop over
+// B x d x d sits on the path.  Every mbarrier wait is bounded (the layout's
+// status word records a wait that ran out).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace bsbr {
+
+constexpr uint32_t kSuspendHintNs = 1000000;   // longest single suspension inside a wait
+
+// ---------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
+// Slow path of a bounded wait: poll (each try suspends the thread for up to
+// kSuspendHintNs or until the phase completes) until the phase completes, the
+// CTA's abort flag is raised, or `limit_ns` passes; on time-out record the
+// status bit and raise the abort flag.
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       uint32_t* status, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > limit_ns) {
+      *abort_flag = 1;
+      atomicOr(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+struct Ctl {
+  volatile int* abort;   // shared: set once any wait of this CTA ran out
+  uint32_t* status;      // global status word
+  uint64_t timeout_ns;
+  // Bounded wait for the completion of the phase with the given parity.
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, abort, status, timeout_ns);
+  }
+};
+
+// Bounded wait that ignores the abort flag (used while draining on exit).
+__device__ __noinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > limit_ns) return;
+  }
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+// TMA (no multicast anywhere in this library).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
+                                            int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0,
+                                            int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+// One 64-key chunk of K or V (rows r0 .. r0+63 of head h, all d columns) as a
+// single box: the tensor map's third dimension walks the 64-column swizzle
+// atoms, so the box lands as [atom][row][64 columns], the layout the MMA
+// descriptors read.
+template <int HD>
+__device__ __forceinline__ void tma_load_kv(uint32_t dst, const CUtensorMap* m, uint32_t bar, int r0, int h) {
+  if constexpr (HD == 128) tma_load_4d(dst, m, bar, 0, r0, 0, h);
+  else tma_load_3d(dst, m, bar, 0, r0, h);
+}
+// The whole 128-row Q tile as a single box: for B = 64 the box spans two
+// consecutive heads (the two stacked query blocks), for B = 128 one block.
+template <int BLK, int HD>
+__device__ __forceinline__ void tma_load_q(uint32_t dst, const CUtensorMap* m, uint32_t bar, int r0, int h) {
+  if constexpr (HD == 128 && BLK == 64) tma_load_4d(dst, m, bar, 0, r0, h, 0);
+  else if constexpr (HD == 128) tma_load_4d(dst, m, bar, 0, r0, 0, h);
+  else tma_load_3d(dst, m, bar, 0, r0, h);
+}
+
+// tcgen05 / TMEM
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+// D(tmem) (+)= A(smem desc) * B(smem desc)
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc)
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+// 16 consecutive 32-bit columns (each holding two bf16 values).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* u) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+      : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= uint64_t((addr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+constexpr uint64_t kDrainNs = 200000000ull;
+
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+struct Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  __nv_bfloat16* o;
+  float* F;        // [kv_heads][chunks][d][d]
+  float* H;        // [kv_heads][chunks][d]
+  uint32_t* status;
+  int n, chunks, heads, kv_heads, group;
+  float scale;
+  uint64_t timeout_ns;
+};
+
+// ---------------------------------------------------------------- chunk states
+// One CTA per (key/value head g, chunk c): F_c = K_c^T V_c as one tcgen05
+// product with M along d (A = the K tile read along d, B = the V tile read
+// along d, the reduction over the chunk's tokens; for d = 64 the upper 64
+// rows of M read the neighbouring tile and are never stored), and H_c = the
+// mean of k over the chunk's tokens.  Tokens past n are zero-filled by the
+// tensor map and left out of the mean.
+template <int BLK, int HD>
+struct StateShape {
+  static constexpr int kBox = 64 * HD * 2;                // one 64-token box: [atom][64 rows][64 columns]
+  static constexpr int kTile = BLK * HD * 2;
+  static constexpr int kOffV = kTile;
+  static constexpr int kOffBar = 2 * kTile;
+  static constexpr int kOffMisc = kOffBar + 16;
+  static constexpr int kSmem = kOffMisc + 16;
+  static constexpr uint32_t kIdesc = idesc_bf16(128, HD, 1, 1);
+};
+
+template <int BLK, int HD>
+__global__ void __launch_bounds__(128) bsbr_state_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                         const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using S = StateShape<BLK, HD>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t base = smem_addr(smem_raw);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
+    return;
+  }
+  const int g = blockIdx.x / p.chunks, c = blockIdx.x - g * p.chunks;
+  const uint32_t sK = base, sV = base + S::kOffV;
+  const uint32_t bLoad = base + S::kOffBar, bDone = bLoad + 8;
+  volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem_raw + S::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + S::kOffMisc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Ctl ctl{abort_flag, p.status, p.timeout_ns};
+  const int t0 = c * BLK;
+  const int count = min(BLK, p.n - t0);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bLoad, 1);
+    mbar_init(bDone, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(base + S::kOffMisc, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(bLoad, 2 * S::kTile);
+#pragma unroll
+    for (int b = 0; b < BLK / 64; ++b) {
+      tma_load_kv<HD>(sK + b * S::kBox, &tmK, bLoad, t0 + b * 64, g);
+      tma_load_kv<HD>(sV + b * S::kBox, &tmV, bLoad, t0 + b * 64, g);
+    }
+    if (ctl.wait(bLoad, 0)) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < BLK / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * S::kBox + (kk & 3) * 2048;
+        mma_ss(tmem, sw128_desc(sK + off, 8192, 1024), sw128_desc(sV + off, 8192, 1024), S::kIdesc, kk > 0);
+      }
+      tc_commit(bDone);
+    } else {
+      tc_commit(bDone);
+      wait_drain(bLoad, 0, kDrainNs);
+    }
+  }
+  // H_c: thread x sums column x over the chunk's tokens
+  if (threadIdx.x < HD) {
+    const __nv_bfloat16* kp = p.k + (size_t(g) * p.n + t0) * HD + threadIdx.x;
+    float acc = 0.f;
+    for (int t = 0; t < count; ++t) acc += __bfloat162float(kp[size_t(t) * HD]);
+    p.H[(size_t(g) * p.chunks + c) * HD + threadIdx.x] = acc / float(count);
+  }
+  // F_c: TMEM lane r holds row r (element r of d) of K_c^T V_c
+  const bool ok = __all_sync(0xffffffffu, ctl.wait(bDone, 0));
+  const int r = warp * 32 + lane;
+  if (ok && !*abort_flag) {
+    tc_fence_after();
+    float* out = p.F + ((size_t(g) * p.chunks + c) * HD + (r < HD ? r : 0)) * HD;
+#pragma unroll
+    for (int a = 0; a < HD / 32; ++a) {
+      float v[32];
+      tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + a * 32, v);
+      tmem_wait_ld();
+      if (r < HD) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(out + a * 32 + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ---------------------------------------------------------------- retrieval
+// One CTA per (query head f, chunk c >= 1): R_c = mean of q over the chunk;
+// a_c' = scale <R_c, H_c'> and A = softmax over c' < c; S_c = sum A_c' F_c'
+// in fp32, split into bf16 hi + lo parts (S = hi + lo to 2^-16); then
+// o_t += q_t S_c for the chunk's tokens as two tcgen05 products
+// (M = 128 tile rows, A = the Q tile, B = S read along d), added to the
+// within-chunk output already in o.  For B = 64 the tile's upper 64 rows are
+// the next chunk's queries and are never stored.
+template <int BLK, int HD>
+struct RetrShape {
+  static constexpr int kQBytes = 128 * HD * 2;
+  static constexpr int kAtomQ = 128 * 128;
+  static constexpr int kSBytes = HD * HD * 2;             // one bf16 S part: [atom][HD rows][64 columns]
+  static constexpr int kAtomS = HD * 128;
+  static constexpr int kOffS = kQBytes;                   // hi, then lo
+  static constexpr int kOffR = kOffS + 2 * kSBytes;       // R_c [HD] fp32
+  static constexpr int kOffRed = kOffR + HD * 4;          // block reduction scratch [8]
+  static constexpr int kOffBar = kOffRed + 64;
+  static constexpr int kOffMisc = kOffBar + 16;
+  static constexpr int kOffA = kOffMisc + 16;             // meta weights [chunks] fp32
+  static constexpr uint32_t kIdesc = idesc_bf16(128, HD, 0, 1);
+};
+
+__device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, v, off);
+    v = is_max ? fmaxf(v, o) : v + o;
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int w = 1; w < int(blockDim.x >> 5); ++w) r = is_max ? fmaxf(r, red[w]) : r + red[w];
+  return r;
+}
+
+template <int BLK, int HD>
+__global__ void __launch_bounds__(256) bsbr_retrieve_kernel(const __grid_constant__ CUtensorMap tmQ, const Params p) {
+  using S = RetrShape<BLK, HD>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t base = smem_addr(smem_raw);
+  if (base & 1023u) {
+    if (threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
+    return;
+  }
+  const int per_head = p.chunks - 1;
+  const int f = blockIdx.x / per_head, c = blockIdx.x - f * per_head + 1;
+  const int g = f / p.group;
+  const int t0 = c * BLK;
+  const int count = min(BLK, p.n - t0);
+  const uint32_t sQ = base, sS = base + S::kOffS;
+  float* R = reinterpret_cast<float*>(smem_raw + S::kOffR);
+  float* red = reinterpret_cast<float*>(smem_raw + S::kOffRed);
+  float* A = reinterpret_cast<float*>(smem_raw + S::kOffA);
+  const uint32_t bLoad = base + S::kOffBar, bDone = bLoad + 8;
+  volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem_raw + S::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + S::kOffMisc + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Ctl ctl{abort_flag, p.status, p.timeout_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(bLoad, 1);
+    mbar_init(bDone, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(base + S::kOffMisc, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(bLoad, S::kQBytes);
+    tma_load_q<128, HD>(sQ, &tmQ, bLoad, t0, f);
+  }
+  // R_c
+  if (threadIdx.x < HD) {
+    const __nv_bfloat16* qp = p.q + (size_t(f) * p.n + t0) * HD + threadIdx.x;
+    float acc = 0.f;
+    for (int t = 0; t < count; ++t) acc += __bfloat162float(qp[size_t(t) * HD]);
+    R[threadIdx.x] = acc / float(count);
+  }
+  __syncthreads();
+  // meta scores of the earlier chunks, one warp per chunk
+  const float* Hg = p.H + size_t(g) * p.chunks * HD;
+  for (int cp = warp; cp < c; cp += 8) {
+    float s = 0.f;
+    for (int x = lane; x < HD; x += 32) s = fmaf(R[x], Hg[size_t(cp) * HD + x], s);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) A[cp] = s * p.scale;
+  }
+  __syncthreads();
+  float m = -INFINITY;
+  for (int cp = threadIdx.x; cp < c; cp += blockDim.x) m = fmaxf(m, A[cp]);
+  m = block_reduce(m, red, true);
+  float z = 0.f;
+  for (int cp = threadIdx.x; cp < c; cp += blockDim.x) {
+    const float e = __expf(A[cp] - m);
+    A[cp] = e;
+    z += e;
+  }
+  z = block_reduce(z, red, false);   // its barriers also publish A
+  const float inv = 1.f / z;
+  // S_c: thread owns float4 columns j4 of rows r = threadIdx.x / (HD/4) + k * (256 / (HD/4))
+  constexpr int kV4 = HD / 4;                 // float4 per row
+  constexpr int kRowsPerPass = 256 / kV4;
+  constexpr int kPasses = HD / kRowsPerPass;
+  const int j4 = threadIdx.x % kV4, r0 = threadIdx.x / kV4;
+  float4 acc[kPasses];
+#pragma unroll
+  for (int k = 0; k < kPasses; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float* Fg = p.F + size_t(g) * p.chunks * HD * HD;
+  for (int cp = 0; cp < c; ++cp) {
+    const float w = A[cp] * inv;
+    const float4* src = reinterpret_cast<const float4*>(Fg + size_t(cp) * HD * HD);
+#pragma unroll
+    for (int k = 0; k < kPasses; ++k) {
+      const float4 x = src[(r0 + k * kRowsPerPass) * kV4 + j4];
+      acc[k].x = fmaf(w, x.x, acc[k].x);
+      acc[k].y = fmaf(w, x.y, acc[k].y);
+      acc[k].z = fmaf(w, x.z, acc[k].z);
+      acc[k].w = fmaf(w, x.w, acc[k].w);
+    }
+  }
+  // S as bf16 hi and lo, [K = d rows][N = d columns] in 64-column swizzled atoms
+#pragma unroll
+  for (int k = 0; k < kPasses; ++k) {
+    const int row = r0 + k * kRowsPerPass, col = j4 * 4;
+    const uint32_t off = uint32_t(col >> 6) * S::kAtomS + uint32_t(row) * 128 +
+                         ((uint32_t(((col & 63) >> 3) ^ (row & 7))) << 4) + uint32_t(col & 7) * 2;
+    const float vals[4] = {acc[k].x, acc[k].y, acc[k].z, acc[k].w};
+    float lo[4];
+    __nv_bfloat16 h[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      h[e] = __float2bfloat16_rn(vals[e]);
+      lo[e] = vals[e] - __bfloat162float(h[e]);
+    }
+    const uint32_t hi01 = uint32_t(__bfloat16_as_ushort(h[0])) | (uint32_t(__bfloat16_as_ushort(h[1])) << 16);
+    const uint32_t hi23 = uint32_t(__bfloat16_as_ushort(h[2])) | (uint32_t(__bfloat16_as_ushort(h[3])) << 16);
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sS + off), "r"(hi01), "r"(hi23) : "memory");
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sS + S::kSBytes + off), "r"(pack_bf16(lo[0], lo[1])),
+                 "r"(pack_bf16(lo[2], lo[3]))
+                 : "memory");
+  }
+  fence_proxy_async();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (ctl.wait(bLoad, 0)) {
+      tc_fence_after();
+#pragma unroll
+      for (int part = 0; part < 2; ++part)
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32;
+          mma_ss(tmem, sw128_desc(sQ + ao, 16, 1024),
+                 sw128_desc(sS + part * S::kSBytes + kk * 16 * 128, S::kAtomS, 1024), S::kIdesc,
+                 (part > 0 || kk > 0) ? 1u : 0u);
+        }
+    } else {
+      wait_drain(bLoad, 0, kDrainNs);
+    }
+    tc_commit(bDone);
+  }
+  if (warp < 4) {
+    const bool ok = __all_sync(0xffffffffu, ctl.wait(bDone, 0));
+    const int r = warp * 32 + lane;
+    if (ok && !*abort_flag) {
+      tc_fence_after();
+      __nv_bfloat16* op = p.o + (size_t(f) * p.n + t0 + r) * HD;
+      const bool mine = r < count;
+#pragma unroll
+      for (int a = 0; a < HD / 32; ++a) {
+        float v[32];
+        tmem_ld32(tmem + (uint32_t(warp * 32) << 16) + a * 32, v);
+        tmem_wait_ld();
+        if (mine) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w = *reinterpret_cast<const uint4*>(op + a * 32 + e);
+            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wp[h]));
+              wp[h] = pack_bf16(x.x + v[e + 2 * h], x.y + v[e + 2 * h + 1]);
+            }
+            *reinterpret_cast<uint4*>(op + a * 32 + e) = w;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+}  // namespace bsbr
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+int g_encode_status = BSA_OK;
+std::string g_encode_msg;
+
+int get_encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q{};
+    void* fn = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) {
+      g_encode_status = BSA_ERR_CUDA;
+      g_encode_msg = std::string("cuTensorMapEncodeTiled unavailable: ") + cudaGetErrorString(e);
+      return;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode_status != BSA_OK) return set_error(g_encode_status, g_encode_msg);
+  return BSA_OK;
+}
+
+int encode_tiled(CUtensorMap* m, const void* ptr, cuuint32_t rank, const cuuint64_t* dims,
+                 const cuuint64_t* strides, const cuuint32_t* box) {
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (" + std::to_string(int(r)) + ")");
+  return BSA_OK;
+}
+
+// [slices][n][d] bf16 in boxes of `rows` rows of one slice, landing as
+// [64-column atom][rows][64 columns] (d = 128: the atom is a tensor dimension
+// of stride 128 bytes, so one box holds both atoms).
+int encode_rows(CUtensorMap* m, const void* ptr, int slices, int n, int d, int rows) {
+  const cuuint64_t row = cuuint64_t(d) * 2, slice = cuuint64_t(n) * row;
+  if (d == 128) {
+    const cuuint64_t dims[4] = {64, cuuint64_t(n), 2, cuuint64_t(slices)};
+    const cuuint64_t str[3] = {row, 128, slice};
+    const cuuint32_t box[4] = {64, cuuint32_t(rows), 2, 1};
+    return encode_tiled(m, ptr, 4, dims, str, box);
+  }
+  const cuuint64_t dims[3] = {64, cuuint64_t(n), cuuint64_t(slices)};
+  const cuuint64_t str[2] = {row, slice};
+  const cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
+  return encode_tiled(m, ptr, 3, dims, str, box);
+}
+
+template <typename K>
+int prepare(K kern, int smem, int slot) {
+  static std::mutex mu;
+  static int done[64][8] = {};
+  int dev_id = 0;
+  cudaError_t e = cudaGetDevice(&dev_id);
+  if (e != cudaSuccess || dev_id < 0 || dev_id >= 64) return set_error(BSA_ERR_CUDA, "cannot query the device");
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev_id][slot] < smem) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    done[dev_id][slot] = smem;
+  }
+  return BSA_OK;
+}
+
+template <int BLK, int HD>
+int launch_instance(const void* q, const void* k, const void* v, const bsbr::Params& p, cudaStream_t stream) {
+  using SS = bsbr::StateShape<BLK, HD>;
+  using SR = bsbr::RetrShape<BLK, HD>;
+  constexpr int slot = (BLK == 128 ? 2 : 0) + (HD == 128 ? 1 : 0);
+  auto ks = bsbr::bsbr_state_kernel<BLK, HD>;
+  auto kr = bsbr::bsbr_retrieve_kernel<BLK, HD>;
+  // no more than four CTAs per SM, so each one's 128 TMEM columns are free at once
+  const int floor_bytes = 46 * 1024;
+  const int smem_s = SS::kSmem > floor_bytes ? SS::kSmem : floor_bytes;
+  const int need_r = SR::kOffA + 4 * p.chunks;
+  const int smem_r = need_r > floor_bytes ? need_r : floor_bytes;
+  if (smem_r > 227 * 1024) return set_error(BSA_ERR_SHAPE, "too many chunks for the retrieval kernel's weights");
+  int st = prepare(ks, smem_s, slot);
+  if (st == BSA_OK) st = prepare(kr, smem_r, 4 + slot);
+  if (st != BSA_OK) return st;
+  CUtensorMap mq, mk, mv;
+  std::memset(&mq, 0, sizeof(mq));
+  std::memset(&mk, 0, sizeof(mk));
+  std::memset(&mv, 0, sizeof(mv));
+  st = encode_rows(&mq, q, p.heads, p.n, HD, 128);
+  if (st == BSA_OK) st = encode_rows(&mk, k, p.kv_heads, p.n, HD, 64);
+  if (st == BSA_OK) st = encode_rows(&mv, v, p.kv_heads, p.n, HD, 64);
+  if (st != BSA_OK) return st;
+  ks<<<p.kv_heads * p.chunks, 128, smem_s, stream>>>(mk, mv, p);
+  kr<<<p.heads * (p.chunks - 1), 256, smem_r, stream>>>(mq, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
+  return BSA_OK;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" size_t bsa_bsbr_workspace_bytes(int n, int B, int kv_heads, int d) {
+  if (n < 1 || B < 1 || kv_heads < 1 || d < 1) return 0;
+  const size_t chunks = size_t((int64_t(n) + B - 1) / B);
+  return size_t(kv_heads) * chunks * size_t(d) * size_t(d + 1) * sizeof(float);
+}
+
+extern "C" int bsa_bsbr_retrieval(const void* q, const void* k, const void* v, const bsa_layout* layout, int B,
+                                  int n, int heads, int kv_heads, int d, float scale, void* o, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  using namespace bsa;
+  if (!layout) return set_error(BSA_ERR_INVALID_ARG, "layout is NULL");
+  if (layout->device < 0 || !layout->d_base)
+    return set_error(BSA_ERR_INVALID_ARG, "layout was built host-only (device = -1)");
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (cur != layout->device) return set_error(BSA_ERR_INVALID_ARG, "layout lives on another device");
+  if (B != layout->B || n != layout->n) return set_error(BSA_ERR_SHAPE, "B/n differ from the layout's");
+  if (B != 64 && B != 128) return set_error(BSA_ERR_UNSUPPORTED, "B must be 64 or 128");
+  if (d != 64 && d != 128) return set_error(BSA_ERR_UNSUPPORTED, "d must be 64 or 128");
+  if (heads < 1 || kv_heads < 1) return set_error(BSA_ERR_SHAPE, "heads and kv_heads must be >= 1");
+  if (heads % kv_heads) return set_error(BSA_ERR_SHAPE, "heads must be a multiple of kv_heads");
+  if (!(std::isfinite(scale) && scale > 0.f)) return set_error(BSA_ERR_INVALID_ARG, "scale must be finite and > 0");
+  if (!q || !k || !v || !o || !workspace) return set_error(BSA_ERR_INVALID_ARG, "null pointer");
+  auto aligned = [](const void* ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; };
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(workspace, 16))
+    return set_error(BSA_ERR_INVALID_ARG, "q, k, v, o and workspace must be 16-byte aligned");
+  if (workspace_bytes < bsa_bsbr_workspace_bytes(n, B, kv_heads, d))
+    return set_error(BSA_ERR_SHAPE, "workspace smaller than bsa_bsbr_workspace_bytes");
+  const int64_t chunks = (int64_t(n) + B - 1) / B;
+  if (int64_t(heads) * chunks > INT32_MAX) return set_error(BSA_ERR_SHAPE, "too many (head, chunk) items");
+  if (chunks < 2) return BSA_OK;   // one chunk: nothing to retrieve
+  int st = get_encoder();
+  if (st != BSA_OK) return st;
+  bsbr::Params p{};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.F = static_cast<float*>(workspace);
+  p.H = p.F + size_t(kv_heads) * size_t(chunks) * d * d;
+  p.status = layout->d_status;
+  p.n = n;
+  p.chunks = int(chunks);
+  p.heads = heads;
+  p.kv_heads = kv_heads;
+  p.group = heads / kv_heads;
+  p.scale = scale;
+  p.timeout_ns = 1000000000ull;   // 1 s: never reached in a correct run
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 64 && d == 128) return launch_instance<64, 128>(q, k, v, p, s);
+  if (B == 64 && d == 64) return launch_instance<64, 64>(q, k, v, p, s);
+  if (B == 128 && d == 128) return launch_instance<128, 128>(q, k, v, p, s);
+  return launch_instance<128, 64>(q, k, v, p, s);
+}

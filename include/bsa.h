@@ -1,6 +1,7 @@
 /*
  * bsa.h -- C ABI of the B200 (sm_100a) block-sparse causal attention
- * forward, its gradients and selected-page decode.
+ * forward, its gradients, selected-page decode and BSBR's between-chunk
+ * retrieval term.
  *
  * What the library computes ("Block-Sparse Attention", ai-model-reference,
  * sections "How It Works" and "Math Or Compute Schema"): the sequence of n
@@ -32,6 +33,7 @@
 #ifndef BSA_H
 #define BSA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -238,6 +240,34 @@ int bsa_backward(const void* q, const void* k, const void* v, const void* o,
                  const float* lse, const void* dout, const bsa_layout* layout,
                  int B, int n, int heads, int kv_heads, int d, float scale,
                  float* dq, float* dk, float* dv, float* workspace, void* stream);
+
+/* Bytes of device workspace bsa_bsbr_retrieval needs: the chunk states
+ * (kv_heads x chunks x d x d fp32) and meta keys (kv_heads x chunks x d fp32),
+ * chunks = ceil(n / B).  0 for sizes < 1. */
+size_t bsa_bsbr_workspace_bytes(int n, int B, int kv_heads, int d);
+
+/* BSBR's between-chunk retrieval term ("bsbr", jvboid.dev/projects/bsbr,
+ * section "Solution"), added to o in place.  Chunks are the layout's blocks of
+ * B tokens.  With R_c, H_c the means of q[f] and k[g] over chunk c (g = f /
+ * (heads / kv_heads)) and F_c = sum over the chunk's tokens of k_u^T v_u:
+ *   A_cc' = softmax over c' < c of scale <R_c, H_c'>,   S_c = sum_{c' < c} A_cc' F_c',
+ *   o[f][t] += q[f][t] S_c   for every token t of chunk c >= 1
+ * (chunk 0 retrieves nothing).  Called after bsa_forward with a
+ * block-diagonal layout (BAND_GLOBAL, window 0, no global block), o becomes
+ * the whole BSBR attention output; lse stays the within-chunk term's.
+ * Layouts: q, o [heads][n][d] bf16; k, v [kv_heads][n][d] bf16; workspace
+ * device memory of at least bsa_bsbr_workspace_bytes.  The layout supplies
+ * the device, B, n and the status word (its kept blocks are not read).
+ * Requirements (checked before launch): layout on the current device and
+ * built for this n and B; B in {64, 128}; d in {64, 128}; heads a multiple of
+ * kv_heads; scale finite and > 0; q, k, v, o, workspace 16-byte aligned and
+ * workspace_bytes large enough.  Enqueues two kernels (none for a single
+ * chunk) and returns; no allocation.  The retrieval costs O(chunks^2 d^2)
+ * per head (each chunk sums the states of all earlier chunks). */
+int bsa_bsbr_retrieval(const void* q, const void* k, const void* v,
+                       const bsa_layout* layout, int B, int n, int heads,
+                       int kv_heads, int d, float scale, void* o,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* Read-only host view of the key/value-gradient work list: for layout head
  * h, segments seg_ptr[h] .. seg_ptr[h+1] - 1, segment s being the triple

@@ -30,7 +30,7 @@ def lib():
 def _declared_functions():
     text = open(os.path.join(ROOT, "include", "bsa.h")).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|void|const char\*)\s+(bsa_\w+)\s*\(", text, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:int|void|size_t|const char\*)\s+(bsa_\w+)\s*\(", text, flags=re.M)))
 
 
 def test_exports_every_declared_symbol(lib):

@@ -7,9 +7,10 @@ full 32K dyadic geometry.
 Tolerance.  The kernels form S and dP exactly in fp32 from the bf16 inputs
 and rebuild P in fp32 from the forward's lse; the products that produce the
 gradients take P and dS = P (dP - D) rounded to bf16 (relative error at most
-2^-9 per term), and D uses the forward's bf16 o.  Each gradient element is a
-sum of such terms, so its error is at most about 2^-9 of the sum of the
-terms' magnitudes.  The test asks for a normwise relative error
+2^-8 per term, bf16's unit roundoff), and D uses the forward's bf16 o.  Each
+gradient element is a sum of such terms, so its error is at most about 2^-8
+of the sum of the terms' magnitudes; with independent rounding the normwise
+error is far smaller (about 1.7e-3 is measured).  The test asks for a normwise relative error
 ||g - g_ref|| / ||g_ref|| <= 1e-2 and max |g - g_ref| <= 2e-2 max |g_ref|
 on each of dq, dk, dv.
 """
