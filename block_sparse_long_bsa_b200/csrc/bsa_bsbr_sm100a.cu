@@ -269,9 +269,38 @@ struct StateShape {
   static constexpr int kOffV = kTile;
   static constexpr int kOffBar = 2 * kTile;
   static constexpr int kOffMisc = kOffBar + 16;
-  static constexpr int kSmem = kOffMisc + 16;
+  static constexpr int kOffRed = kOffMisc + 16;            // [128] partial column sums
+  static constexpr int kSmem = kOffRed + 128 * 4;
   static constexpr uint32_t kIdesc = idesc_bf16(128, HD, 1, 1);
 };
+
+// Element (row t, column x) of a bf16 tile landed by the tensor maps as
+// [64-row box][64-column atom][row][128-byte swizzled line].
+template <int HD>
+__device__ __forceinline__ float tile_elem(const uint8_t* tile, int rows_per_box, int t, int x) {
+  const int box = t / rows_per_box, row = t - box * rows_per_box;
+  const int off = box * rows_per_box * HD * 2 + (x >> 6) * rows_per_box * 128 + row * 128 +
+                  ((((x & 63) >> 3) ^ (row & 7)) << 4) + (x & 7) * 2;
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
+}
+
+// Column means of the first `count` rows of a tile in shared memory, by all
+// threads of the block (blockDim.x a multiple of HD); out[x] for x < HD.
+template <int HD>
+__device__ __forceinline__ void tile_column_means(const uint8_t* tile, int rows_per_box, int count, float* part,
+                                                  float* out) {
+  const int groups = int(blockDim.x) / HD;
+  const int x = threadIdx.x % HD, gr = threadIdx.x / HD;
+  float acc = 0.f;
+  for (int t = gr; t < count; t += groups) acc += tile_elem<HD>(tile, rows_per_box, t, x);
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.x < HD) {
+    float sum = 0.f;
+    for (int k = 0; k < groups; ++k) sum += part[k * HD + threadIdx.x];
+    out[threadIdx.x] = sum / float(count);
+  }
+}
 
 template <int BLK, int HD>
 __global__ void __launch_bounds__(128) bsbr_state_kernel(const __grid_constant__ CUtensorMap tmK,
@@ -315,26 +344,25 @@ __global__ void __launch_bounds__(128) bsbr_state_kernel(const __grid_constant__
       tma_load_kv<HD>(sK + b * S::kBox, &tmK, bLoad, t0 + b * 64, g);
       tma_load_kv<HD>(sV + b * S::kBox, &tmV, bLoad, t0 + b * 64, g);
     }
-    if (ctl.wait(bLoad, 0)) {
+  }
+  const bool loaded = __syncthreads_and(ctl.wait(bLoad, 0));
+  if (threadIdx.x == 0) {
+    if (loaded) {
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < BLK / 16; ++kk) {
         const uint32_t off = (kk >> 2) * S::kBox + (kk & 3) * 2048;
         mma_ss(tmem, sw128_desc(sK + off, 8192, 1024), sw128_desc(sV + off, 8192, 1024), S::kIdesc, kk > 0);
       }
-      tc_commit(bDone);
     } else {
-      tc_commit(bDone);
       wait_drain(bLoad, 0, kDrainNs);
     }
+    tc_commit(bDone);
   }
-  // H_c: thread x sums column x over the chunk's tokens
-  if (threadIdx.x < HD) {
-    const __nv_bfloat16* kp = p.k + (size_t(g) * p.n + t0) * HD + threadIdx.x;
-    float acc = 0.f;
-    for (int t = 0; t < count; ++t) acc += __bfloat162float(kp[size_t(t) * HD]);
-    p.H[(size_t(g) * p.chunks + c) * HD + threadIdx.x] = acc / float(count);
-  }
+  // H_c: column means of the K tile
+  if (loaded)
+    tile_column_means<HD>(smem_raw, 64, count, reinterpret_cast<float*>(smem_raw + S::kOffRed),
+                          p.H + (size_t(g) * p.chunks + c) * HD);
   // F_c: TMEM lane r holds row r (element r of d) of K_c^T V_c
   const bool ok = __all_sync(0xffffffffu, ctl.wait(bDone, 0));
   const int r = warp * 32 + lane;
@@ -378,7 +406,8 @@ struct RetrShape {
   static constexpr int kOffS = kQBytes;                   // hi, then lo
   static constexpr int kOffR = kOffS + 2 * kSBytes;       // R_c [HD] fp32
   static constexpr int kOffRed = kOffR + HD * 4;          // block reduction scratch [8]
-  static constexpr int kOffBar = kOffRed + 64;
+  static constexpr int kOffPart = kOffRed + 64;           // [256] partial column sums
+  static constexpr int kOffBar = kOffPart + 256 * 4;
   static constexpr int kOffMisc = kOffBar + 16;
   static constexpr int kOffA = kOffMisc + 16;             // meta weights [chunks] fp32
   static constexpr uint32_t kIdesc = idesc_bf16(128, HD, 0, 1);
@@ -441,22 +470,30 @@ __global__ void __launch_bounds__(256) bsbr_retrieve_kernel(const __grid_constan
     mbar_expect_tx(bLoad, S::kQBytes);
     tma_load_q<128, HD>(sQ, &tmQ, bLoad, t0, f);
   }
-  // R_c
-  if (threadIdx.x < HD) {
-    const __nv_bfloat16* qp = p.q + (size_t(f) * p.n + t0) * HD + threadIdx.x;
-    float acc = 0.f;
-    for (int t = 0; t < count; ++t) acc += __bfloat162float(qp[size_t(t) * HD]);
-    R[threadIdx.x] = acc / float(count);
-  }
+  // R_c: column means of the Q tile (one 128-row box)
+  const bool loaded = __syncthreads_and(ctl.wait(bLoad, 0));
+  if (loaded) tile_column_means<HD>(smem_raw, 128, count, reinterpret_cast<float*>(smem_raw + S::kOffPart), R);
   __syncthreads();
-  // meta scores of the earlier chunks, one warp per chunk
+  // meta scores of the earlier chunks, one warp per chunk, four chunks' loads in flight
   const float* Hg = p.H + size_t(g) * p.chunks * HD;
-  for (int cp = warp; cp < c; cp += 8) {
-    float s = 0.f;
-    for (int x = lane; x < HD; x += 32) s = fmaf(R[x], Hg[size_t(cp) * HD + x], s);
+  for (int cp0 = warp; cp0 < c; cp0 += 32) {
+    float sc[4];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) A[cp] = s * p.scale;
+    for (int u = 0; u < 4; ++u) {
+      const int cp = cp0 + 8 * u;
+      float s = 0.f;
+      if (cp < c) {
+#pragma unroll
+        for (int x = lane; x < HD; x += 32) s = fmaf(R[x], Hg[size_t(cp) * HD + x], s);
+      }
+      sc[u] = s;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], off);
+      if (lane == 0 && cp0 + 8 * u < c) A[cp0 + 8 * u] = sc[u] * p.scale;
+    }
   }
   __syncthreads();
   float m = -INFINITY;
@@ -479,16 +516,27 @@ __global__ void __launch_bounds__(256) bsbr_retrieve_kernel(const __grid_constan
 #pragma unroll
   for (int k = 0; k < kPasses; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   const float* Fg = p.F + size_t(g) * p.chunks * HD * HD;
-  for (int cp = 0; cp < c; ++cp) {
-    const float w = A[cp] * inv;
-    const float4* src = reinterpret_cast<const float4*>(Fg + size_t(cp) * HD * HD);
+  // U earlier states per step, their loads issued together
+  constexpr int U = HD == 64 ? 4 : 2;
+  for (int cp0 = 0; cp0 < c; cp0 += U) {
+    float4 x[U][kPasses];
 #pragma unroll
-    for (int k = 0; k < kPasses; ++k) {
-      const float4 x = src[(r0 + k * kRowsPerPass) * kV4 + j4];
-      acc[k].x = fmaf(w, x.x, acc[k].x);
-      acc[k].y = fmaf(w, x.y, acc[k].y);
-      acc[k].z = fmaf(w, x.z, acc[k].z);
-      acc[k].w = fmaf(w, x.w, acc[k].w);
+    for (int u = 0; u < U; ++u) {
+      const int cp = cp0 + u < c ? cp0 + u : c - 1;
+      const float4* src = reinterpret_cast<const float4*>(Fg + size_t(cp) * HD * HD);
+#pragma unroll
+      for (int k = 0; k < kPasses; ++k) x[u][k] = src[(r0 + k * kRowsPerPass) * kV4 + j4];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const float w = cp0 + u < c ? A[cp0 + u] * inv : 0.f;
+#pragma unroll
+      for (int k = 0; k < kPasses; ++k) {
+        acc[k].x = fmaf(w, x[u][k].x, acc[k].x);
+        acc[k].y = fmaf(w, x[u][k].y, acc[k].y);
+        acc[k].z = fmaf(w, x[u][k].z, acc[k].z);
+        acc[k].w = fmaf(w, x[u][k].w, acc[k].w);
+      }
     }
   }
   // S as bf16 hi and lo, [K = d rows][N = d columns] in 64-column swizzled atoms
@@ -515,7 +563,7 @@ __global__ void __launch_bounds__(256) bsbr_retrieve_kernel(const __grid_constan
   fence_proxy_async();
   __syncthreads();
   if (threadIdx.x == 0) {
-    if (ctl.wait(bLoad, 0)) {
+    if (loaded) {
       tc_fence_after();
 #pragma unroll
       for (int part = 0; part < 2; ++part)

@@ -11,12 +11,14 @@
 // P is rebuilt from the forward's lse, so no n x n matrix is stored.
 //
 // Three launches on the caller's stream: D (one warp per row), then the dq
-// kernel (one CTA per query tile, walking the tile's CSR row of kept blocks)
-// and the dk/dv kernel (one CTA per segment of a key block's column of the
-// transposed layout, walking the query tiles that read it).  Both product
-// kernels use 160 threads: warp 0 issues the TMA loads and, from one thread,
-// the tcgen05 products; warps 1-4 hold one tile row per thread (warp w reaches
-// TMEM lanes 32 (w % 4) ..) and rebuild P and dS.  Every product is a
+// kernel (query tiles, each walking its CSR row of kept blocks) and the dk/dv
+// kernel (segments of a key block's column of the transposed layout, each
+// walking the query tiles that read it).  Both product kernels are
+// persistent, one CTA per SM, 192 threads: warp 0 issues the TMA loads; one
+// thread of warp 1 issues the tcgen05 products, each as soon as its inputs
+// are ready (two kinds of product interleave, so neither waits behind the
+// other); warps 2-5 hold one tile row per thread (warp w reaches TMEM lanes
+// 32 (w % 4) ..) and rebuild P and dS.  Every product is a
 // 128-row bf16 x bf16 -> fp32 tcgen05 MMA accumulating in TMEM.  Every
 // mbarrier wait is bounded: one that runs out sets the layout's status word,
 // the CTA drains what it has in flight, releases TMEM and returns.
@@ -58,6 +60,18 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
+}
+// Non-blocking test of a phase (used where one thread watches several barriers).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -242,7 +256,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo_bytes
 }
 
 // ---------------------------------------------------------------- shared
-constexpr int kThreads = 160;        // warp 0: loads and products; warps 1-4: one tile row per thread
+constexpr int kThreads = 192;        // warp 0: loads; warp 1: products; warps 2-5: one tile row per thread
 constexpr int kTileM = 128;          // rows of every product tile (tcgen05 M = 128)
 constexpr int kChunk = 64;           // keys per chunk
 constexpr float kLog2e = 1.4426950408889634f;
@@ -268,7 +282,8 @@ struct Params {
   float* dk;
   float* dv;
   uint32_t* status;
-  int n, nb, L, kv_heads, group, pack, n_steps;   // n_steps = group / pack head steps per key/value head
+  int n, nb, L, heads, kv_heads, group, pack, n_steps;   // n_steps = group / pack head steps per key/value head
+  int items;         // work items of the launched kernel
   float scale, scale_log2;
   uint64_t timeout_ns;
 };
@@ -329,11 +344,15 @@ __global__ void __launch_bounds__(256) bsa_bwd_rowdot_kernel(const __nv_bfloat16
 }
 
 // ---------------------------------------------------------------- dQ
-// One CTA per query tile, tiles longest row first.  Per 64-key chunk c of the
-// tile's kept blocks: S = Q K_c^T and dP = dO V_c^T into TMEM buffer c & 1;
-// the row threads turn them into dS = P (dP - D), rounded to bf16 over the S
-// buffer; then dQ += dS K_c (A = dS read from TMEM, B = K_c read along d).
-// K_c and V_c stay in shared-memory slot c % 3 until dQ_c is done.
+// Persistent: one CTA per SM walks query tiles (longest row first, every
+// gridDim-th).  Per 64-key chunk c of a tile's kept blocks: S = Q K_c^T and
+// dP = dO V_c^T into TMEM buffer c & 1; the row threads turn them into
+// dS = P (dP - D), rounded to bf16 over the S buffer; then dQ += dS K_c
+// (A = dS read from TMEM, B = K_c read along d) into the tile's accumulator
+// (two TMEM accumulators, so one tile's read-out overlaps the next tile's
+// products).  Chunks are numbered across the CTA's tiles: K_c sits in slot
+// c % 4 until dQ_c is done, V_c in slot c % 2 until S_c / dP_c are done, and
+// a tile's Q and dO in buffer (tile & 1) until its last S / dP are done.
 template <int BLK, int HD>
 struct DqShape {
   static constexpr int kCPB = BLK / kChunk;
@@ -341,19 +360,77 @@ struct DqShape {
   static constexpr int kTile = kChunk * HD * 2;
   static constexpr int kAtomQ = kTileM * 128;
   static constexpr int kAtomKV = kChunk * 128;
-  static constexpr int kOffDO = kQBytes;
-  static constexpr int kOffK = 2 * kQBytes;
-  static constexpr int kOffV = kOffK + 3 * kTile;
-  static constexpr int kOffBar = kOffV + 3 * kTile;
-  // q_full, kv_full[3], s_full[2], ds_full[2], dq_done[3], drain
-  static constexpr int kNumBars = 12;
+  static constexpr int kRingK = 4, kRingV = 2;
+  static constexpr int kOffK = 4 * kQBytes;                // Q, dO of buffer b at b * 2 * kQBytes
+  static constexpr int kOffV = kOffK + kRingK * kTile;
+  static constexpr int kOffBar = kOffV + kRingV * kTile;
+  // q_full[2] q_free[2] k_full[4] k_free[4] v_full[2] s_full[2] ds_full[2] acc_full[2] acc_free[2] drain
+  static constexpr int kBQ = 0, kBQFree = 2, kBK = 4, kBKFree = 8, kBV = 12, kBS = 14, kBDS = 16, kBAcc = 18,
+                       kBAccFree = 20, kBDrain = 22, kNumBars = 23;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColQ = 256;
   static constexpr uint32_t kIdescS = idesc_bf16(kTileM, kChunk, 0, 0);
   static constexpr uint32_t kIdescDQ = idesc_bf16(kTileM, HD, 0, 1);
-  static_assert(4 * 32 * 33 * 4 <= 3 * kTile, "epilogue staging fits the K ring");
+  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static_assert(kColQ + 2 * HD <= 512, "TMEM columns");
 };
+
+struct DqItem {
+  QTile tile;
+  int kvh, start, nch, diag_first;
+};
+
+template <int BLK>
+__device__ __forceinline__ DqItem dq_item(const Params& p, int x) {
+  constexpr int CPB = BLK / kChunk;
+  const int n_hg = p.heads / p.pack;
+  const int rank = x / n_hg, hg = x - rank * n_hg;
+  DqItem it;
+  it.tile.h0 = hg * p.pack;
+  const int lh = it.tile.h0 % p.L;
+  it.tile.i = p.order[size_t(lh) * p.nb + rank];
+  it.kvh = it.tile.h0 / p.group;
+  const size_t lrow = size_t(lh) * p.nb + it.tile.i;
+  it.start = p.row_ptr[lrow];
+  const int len = p.row_ptr[lrow + 1] - it.start;
+  it.nch = len * CPB;
+  const bool diag_last = len > 0 && p.col_idx[it.start + len - 1] == it.tile.i;
+  it.diag_first = diag_last ? it.nch - CPB : it.nch;
+  return it;
+}
+
+// A position in a CTA's stream of chunks: item x (global index), chunk c of
+// it, global chunk number g, and the count of non-empty items before it.
+struct DqCursor {
+  int x, c, g, xi;
+  DqItem it;
+  bool valid;
+};
+
+template <int BLK>
+__device__ __forceinline__ void dq_seek(const Params& p, DqCursor& k) {
+  // skip empty items from k.x on
+  while (k.x < p.items) {
+    k.it = dq_item<BLK>(p, k.x);
+    if (k.it.nch > 0) {
+      k.valid = true;
+      return;
+    }
+    k.x += gridDim.x;
+  }
+  k.valid = false;
+}
+
+template <int BLK>
+__device__ __forceinline__ void dq_advance(const Params& p, DqCursor& k) {
+  ++k.g;
+  if (++k.c < k.it.nch) return;
+  k.c = 0;
+  ++k.xi;
+  k.x += gridDim.x;
+  dq_seek<BLK>(p, k);
+}
 
 template <int BLK, int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -361,54 +438,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const Params p) {
   using S = DqShape<BLK, HD>;
+  constexpr int CPB = S::kCPB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_addr(smem_raw);
   if (base & 1023u) {
     if (threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
     return;
   }
-  const uint32_t sQ = base, sDO = base + S::kOffDO, sK = base + S::kOffK, sV = base + S::kOffV;
   const uint32_t bar0 = base + S::kOffBar;
-  const uint32_t bQ = bar0;
-  auto bKV = [&](int c) { return bar0 + 8u * (1 + c % 3); };
-  auto bS = [&](int c) { return bar0 + 8u * (4 + (c & 1)); };
-  auto bDS = [&](int c) { return bar0 + 8u * (6 + (c & 1)); };
-  auto bDQ = [&](int c) { return bar0 + 8u * (8 + c % 3); };
-  const uint32_t bDrain = bar0 + 8u * 11;
+  auto bar = [&](int idx) { return bar0 + 8u * uint32_t(idx); };
+  auto sQ = [&](int b) { return base + uint32_t(b) * 2 * S::kQBytes; };
+  auto sK = [&](int g) { return base + S::kOffK + uint32_t(g % S::kRingK) * S::kTile; };
+  auto sV = [&](int g) { return base + S::kOffV + uint32_t(g % S::kRingV) * S::kTile; };
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem_raw + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + S::kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Ctl ctl{abort_flag, p.status, p.timeout_ns};
 
-  // item -> (rank in the longest-first order, head group): every head
-  // group's longest rows go first
-  const int n_hg = gridDim.x / p.nb;
-  const int rank = blockIdx.x / n_hg, hg = blockIdx.x - rank * n_hg;
-  const int h0 = hg * p.pack;
-  const int lh = h0 % p.L;
-  const QTile tile{p.order[size_t(lh) * p.nb + rank], h0};
-  const int kvh = h0 / p.group;
-  const size_t lrow = size_t(lh) * p.nb + tile.i;
-  const int start = p.row_ptr[lrow], len = p.row_ptr[lrow + 1] - start;
-  const bool diag_last = len > 0 && p.col_idx[start + len - 1] == tile.i;
-  const int nch = len * S::kCPB;
-  const int diag_first = diag_last ? nch - S::kCPB : nch;
-
   if (threadIdx.x == 0) {
-    mbar_init(bQ, 1);
-    for (int s = 0; s < 3; ++s) {
-      mbar_init(bar0 + 8u * (1 + s), 1);
-      mbar_init(bar0 + 8u * (8 + s), 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar0 + 8u * (4 + s), 1);
-      mbar_init(bar0 + 8u * (6 + s), 128);
-    }
-    mbar_init(bDrain, 1);
+    for (int b = 0; b < S::kNumBars; ++b)
+      mbar_init(bar(b), (b == S::kBDS || b == S::kBDS + 1 || b == S::kBAccFree || b == S::kBAccFree + 1) ? 128u : 1u);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(base + S::kOffMisc, 512);
     tmem_relinquish();
   }
@@ -418,147 +471,199 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
-    if (lane == 0 && nch > 0) {
+    // ---- loads
+    if (lane == 0) {
       bool ok = true;
-      int loaded = 0;
-      auto key0 = [&](int c) { return p.col_idx[start + c / S::kCPB] * BLK + (c % S::kCPB) * kChunk; };
-      auto load = [&](int c) -> bool {
-        if (c >= 3 && !ctl.wait(bDQ(c), uint32_t((c - 3) / 3) & 1u)) return false;   // dQ_{c-3} done
-        mbar_expect_tx(bKV(c), 2 * S::kTile);
-        const uint32_t slot = uint32_t(c % 3) * S::kTile;
-        const int k0 = key0(c);
-        tma_load_kv<HD>(sK + slot, &tmK, bKV(c), k0, kvh);
-        tma_load_kv<HD>(sV + slot, &tmV, bKV(c), k0, kvh);
-        ++loaded;
-        return true;
-      };
-      auto products_s = [&](int c) -> bool {
-        if (!ctl.wait(bKV(c), uint32_t(c / 3) & 1u)) return false;
-        tc_fence_after();
-        const uint32_t slot = uint32_t(c % 3) * S::kTile;
-        const uint32_t ds = tmem + S::kColS + (c & 1) * kChunk, ddp = tmem + S::kColDP + (c & 1) * kChunk;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
-          mma_ss(ds, sw128_desc(sQ + ao, 16, 1024), sw128_desc(sK + slot + bo, 16, 1024), S::kIdescS, kk > 0);
-          mma_ss(ddp, sw128_desc(sDO + ao, 16, 1024), sw128_desc(sV + slot + bo, 16, 1024), S::kIdescS, kk > 0);
+      int nk = 0, nv = 0, xi = 0;   // K, V and Q / dO loads issued (chunk g's K is load g)
+      for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
+        const DqItem it = dq_item<BLK>(p, x);
+        if (it.nch == 0) continue;
+        const int b = xi & 1;
+        if (xi >= 2 && !(ok = ctl.wait(bar(S::kBQFree + b), uint32_t((xi - 2) >> 1) & 1u))) break;
+        mbar_expect_tx(bar(S::kBQ + b), 2 * S::kQBytes);
+        tma_load_q<BLK, HD>(sQ(b), &tmQ, bar(S::kBQ + b), it.tile.i * BLK, it.tile.h0);
+        tma_load_q<BLK, HD>(sQ(b) + S::kQBytes, &tmDO, bar(S::kBQ + b), it.tile.i * BLK, it.tile.h0);
+        ++xi;
+        for (int c = 0; c < it.nch; ++c) {
+          const int g = nk;
+          const int key0 = p.col_idx[it.start + c / CPB] * BLK + (c % CPB) * kChunk;
+          // K slot g % 4 held chunk g - 4 until its dQ product; V slot g % 2
+          // held chunk g - 2 until its S / dP products
+          if (g >= S::kRingK && !(ok = ctl.wait(bar(S::kBKFree + g % S::kRingK), uint32_t((g - S::kRingK) / S::kRingK) & 1u)))
+            break;
+          mbar_expect_tx(bar(S::kBK + g % S::kRingK), S::kTile);
+          tma_load_kv<HD>(sK(g), &tmK, bar(S::kBK + g % S::kRingK), key0, it.kvh);
+          ++nk;
+          if (g >= S::kRingV && !(ok = ctl.wait(bar(S::kBS + (g & 1)), uint32_t((g - S::kRingV) >> 1) & 1u))) break;
+          mbar_expect_tx(bar(S::kBV + g % S::kRingV), S::kTile);
+          tma_load_kv<HD>(sV(g), &tmV, bar(S::kBV + g % S::kRingV), key0, it.kvh);
+          ++nv;
         }
-        tc_commit(bS(c));
-        return true;
-      };
-      auto product_dq = [&](int c) -> bool {
-        if (!ctl.wait(bDS(c), uint32_t(c >> 1) & 1u)) return false;
-        tc_fence_after();
-        const uint32_t slot = uint32_t(c % 3) * S::kTile;
-        const uint32_t pa = tmem + S::kColS + (c & 1) * kChunk;
-#pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk)
-          mma_ts(tmem + S::kColQ, pa + kk * 8, sw128_desc(sK + slot + kk * 16 * 128, S::kAtomKV, 1024), S::kIdescDQ,
-                 (c > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bDQ(c));
-        return true;
-      };
-      mbar_expect_tx(bQ, 2 * S::kQBytes);
-      tma_load_q<BLK, HD>(sQ, &tmQ, bQ, tile.i * BLK, tile.h0);
-      tma_load_q<BLK, HD>(sDO, &tmDO, bQ, tile.i * BLK, tile.h0);
-      for (int c = 0; c < nch && c < 3 && ok; ++c) ok = load(c);
-      if (ok) ok = ctl.wait(bQ, 0);
-      if (ok) ok = products_s(0);
-      if (ok && nch > 1) ok = products_s(1);
-      for (int c = 0; c < nch && ok; ++c) {
-        ok = product_dq(c);
-        if (ok && c + 2 < nch) ok = products_s(c + 2);
-        if (ok && c + 3 < nch) ok = load(c + 3);
       }
-      tc_commit(bDrain);
-      wait_drain(bDrain, 0, kDrainNs);
-      wait_drain(bQ, 0, kDrainNs);
-      for (int c = (loaded > 3 ? loaded - 3 : 0); c < loaded; ++c) wait_drain(bKV(c), uint32_t(c / 3) & 1u, kDrainNs);
+      if (!ok) {
+        // let the copies in flight land before the CTA exits
+        for (int e = (nk > S::kRingK ? nk - S::kRingK : 0); e < nk; ++e)
+          wait_drain(bar(S::kBK + e % S::kRingK), uint32_t(e / S::kRingK) & 1u, kDrainNs);
+        for (int e = (nv > S::kRingV ? nv - S::kRingV : 0); e < nv; ++e)
+          wait_drain(bar(S::kBV + e % S::kRingV), uint32_t(e / S::kRingV) & 1u, kDrainNs);
+        for (int e = (xi > 2 ? xi - 2 : 0); e < xi; ++e) wait_drain(bar(S::kBQ + (e & 1)), uint32_t(e >> 1) & 1u, kDrainNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- products, issued as their inputs become ready
+    if (lane == 0) {
+      DqCursor cs{int(blockIdx.x), 0, 0, 0, {}, false}, cd{int(blockIdx.x), 0, 0, 0, {}, false};
+      dq_seek<BLK>(p, cs);
+      dq_seek<BLK>(p, cd);
+      uint64_t idle_since = 0;
+      bool ok = true;
+      while (cd.valid && ok) {
+        bool progress = false;
+        if (cs.valid && cs.g < cd.g + 2 && mbar_test(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u) &&
+            mbar_test(bar(S::kBK + cs.g % S::kRingK), uint32_t(cs.g / S::kRingK) & 1u) &&
+            mbar_test(bar(S::kBV + cs.g % S::kRingV), uint32_t(cs.g / S::kRingV) & 1u)) {
+          tc_fence_after();
+          const uint32_t qb = sQ(cs.xi & 1), kb = sK(cs.g), vb = sV(cs.g);
+          const uint32_t ds = tmem + S::kColS + (cs.g & 1) * kChunk, ddp = tmem + S::kColDP + (cs.g & 1) * kChunk;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
+            mma_ss(ds, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
+            mma_ss(ddp, sw128_desc(qb + S::kQBytes + ao, 16, 1024), sw128_desc(vb + bo, 16, 1024), S::kIdescS,
+                   kk > 0);
+          }
+          tc_commit(bar(S::kBS + (cs.g & 1)));
+          if (cs.c == cs.it.nch - 1) tc_commit(bar(S::kBQFree + (cs.xi & 1)));
+          dq_advance<BLK>(p, cs);
+          progress = true;
+        }
+        if (cd.g < cs.g || !cs.valid) {
+          if (mbar_test(bar(S::kBDS + (cd.g & 1)), uint32_t(cd.g >> 1) & 1u) &&
+              (cd.c > 0 || cd.xi < 2 ||
+               mbar_test(bar(S::kBAccFree + (cd.xi & 1)), uint32_t((cd.xi - 2) >> 1) & 1u))) {
+            tc_fence_after();
+            const uint32_t pa = tmem + S::kColS + (cd.g & 1) * kChunk, kb = sK(cd.g);
+            const uint32_t acc = tmem + S::kColQ + uint32_t(cd.xi & 1) * HD;
+#pragma unroll
+            for (int kk = 0; kk < kChunk / 16; ++kk)
+              mma_ts(acc, pa + kk * 8, sw128_desc(kb + kk * 16 * 128, S::kAtomKV, 1024), S::kIdescDQ,
+                     (cd.c > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(bar(S::kBKFree + cd.g % S::kRingK));
+            if (cd.c == cd.it.nch - 1) tc_commit(bar(S::kBAcc + (cd.xi & 1)));
+            dq_advance<BLK>(p, cd);
+            progress = true;
+          }
+        }
+        if (progress) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer();
+          if (idle_since == 0) idle_since = now;
+          if (*abort_flag) ok = false;
+          else if (now - idle_since > p.timeout_ns) {
+            *abort_flag = 1;
+            atomicOr(p.status, kStatusTimeout);
+            ok = false;
+          }
+        }
+      }
+      tc_commit(bar(S::kBDrain));
+      wait_drain(bar(S::kBDrain), 0, kDrainNs);
     }
   } else {
+    // ---- rows: dS, then each tile's dQ read-out
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
-    int head, tok;
-    const bool real = tile_row<BLK>(p, tile, r, head, tok);
     const int rl = r - (r / BLK) * BLK;
-    const size_t rowi = size_t(head) * p.n + (real ? tok : 0);
-    const float lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
-    const float dd = real ? p.dsum[rowi] : 0.f;
-    const bool live = real && lse2 > -INFINITY;
     bool ok = true;
-    for (int c = 0; c < nch && ok; ++c) {
-      ok = __all_sync(0xffffffffu, ctl.wait(bS(c), uint32_t(c >> 1) & 1u));
+    int g = 0, xi = 0;
+    for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
+      const DqItem it = dq_item<BLK>(p, x);
+      int head, tok;
+      const bool real = tile_row<BLK>(p, it.tile, r, head, tok);
+      const size_t rowi = size_t(head) * p.n + (real ? tok : 0);
+      float* out = p.dq + rowi * HD;
+      if (it.nch == 0) {
+        if (real) {
+#pragma unroll
+          for (int e = 0; e < HD; e += 4) *reinterpret_cast<float4*>(out + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        continue;
+      }
+      const float lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
+      const float dd = real ? p.dsum[rowi] : 0.f;
+      const bool live = real && lse2 > -INFINITY;
+      for (int c = 0; c < it.nch; ++c, ++g) {
+        ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBS + (g & 1)), uint32_t(g >> 1) & 1u));
+        if (!ok) break;
+        tc_fence_after();
+        float s[kChunk], dp[kChunk], pv[kChunk];
+        const uint32_t cs = lane_base + S::kColS + (g & 1) * kChunk, cdp = lane_base + S::kColDP + (g & 1) * kChunk;
+        tmem_ld32(cs, s);
+        tmem_ld32(cs + 32, s + 32);
+        tmem_ld32(cdp, dp);
+        tmem_ld32(cdp + 32, dp + 32);
+        tmem_wait_ld();
+        const int lim = c >= it.diag_first ? rl - (c - it.diag_first) * kChunk : kChunk;
+        p_ds_row(s, dp, pv, p.scale_log2, lse2, dd, lim, live);
+#pragma unroll
+        for (int h = 0; h < kChunk / 32; ++h) {
+          uint32_t u[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(s[h * 32 + 2 * e], s[h * 32 + 2 * e + 1]);
+          tmem_st16(cs + h * 16, u);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(S::kBDS + (g & 1)));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBAcc + (xi & 1)), uint32_t(xi >> 1) & 1u));
       if (!ok) break;
       tc_fence_after();
-      float s[kChunk], dp[kChunk], pv[kChunk];
-      const uint32_t cs = lane_base + S::kColS + (c & 1) * kChunk, cd = lane_base + S::kColDP + (c & 1) * kChunk;
-      tmem_ld32(cs, s);
-      tmem_ld32(cs + 32, s + 32);
-      tmem_ld32(cd, dp);
-      tmem_ld32(cd + 32, dp + 32);
-      tmem_wait_ld();
-      const int lim = c >= diag_first ? rl - (c - diag_first) * kChunk : kChunk;
-      p_ds_row(s, dp, pv, p.scale_log2, lse2, dd, lim, live);
-#pragma unroll
-      for (int h = 0; h < kChunk / 32; ++h) {
-        uint32_t u[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) u[e] = pack_bf16(s[h * 32 + 2 * e], s[h * 32 + 2 * e + 1]);
-        tmem_st16(cs + h * 16, u);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bDS(c));
-    }
-    if (ok && nch > 0) ok = __all_sync(0xffffffffu, ctl.wait(bDQ(nch - 1), uint32_t((nch - 1) / 3) & 1u));
-    if (ok) {
-      // dQ = scale * acc, through a per-warp [32 rows][33] staging tile in the
-      // (idle) K ring so each row is written as whole 128-byte lines
-      tc_fence_after();
-      float* stage = reinterpret_cast<float*>(smem_raw + S::kOffK) + q4 * 32 * 33;
-      const int row0 = q4 * 32;
+      const uint32_t acc = lane_base + S::kColQ + uint32_t(xi & 1) * HD;
 #pragma unroll 1
       for (int a = 0; a < HD / 32; ++a) {
         float v[32];
-        if (nch > 0) {
-          tmem_ld32(lane_base + S::kColQ + a * 32, v);
-          tmem_wait_ld();
-        } else {
+        tmem_ld32(acc + a * 32, v);
+        tmem_wait_ld();
+        if (real) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0.f;
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(out + a * 32 + e) =
+                make_float4(v[e] * p.scale, v[e + 1] * p.scale, v[e + 2] * p.scale, v[e + 3] * p.scale);
         }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) stage[lane * 33 + e] = v[e] * p.scale;
-        __syncwarp();
-        for (int rr = 0; rr < 32; ++rr) {
-          int hh, tt;
-          if (tile_row<BLK>(p, tile, row0 + rr, hh, tt))
-            p.dq[(size_t(hh) * p.n + tt) * HD + a * 32 + lane] = stage[rr * 33 + lane];
-        }
-        __syncwarp();
       }
+      tc_fence_before();
+      mbar_arrive(bar(S::kBAccFree + (xi & 1)));
+      ++xi;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
 // ---------------------------------------------------------------- dK, dV
-// One CTA per (key/value head, query-head step, 64-key chunk of a key block,
-// column segment): the segment lists up to 16 query blocks whose rows keep
-// the key block (the transposed layout).  Per query tile t of the segment:
-// S = Q K^T and dP = dO V^T (M = 128 query rows) into TMEM buffer t & 1; the
-// row threads write P and dS = P (dP - D) as bf16 [query][key] tiles into
-// shared-memory buffer t & 1; then dV^T += dO^T P and dK^T += Q^T dS (M = 128
-// along d: A is the dO / Q tile read along d, B the P / dS tile read along
-// the keys; for d = 64 the upper 64 rows of M read the neighbouring tile and
-// are never stored).  The sums are added into dk and dv (zeroed first), as
-// segments of one column run on several CTAs.
+// Persistent: one CTA per SM walks work items (key/value head, query-head
+// step, 64-key chunk of a key block, column segment; longest segments first,
+// every gridDim-th).  A segment lists up to 16 query blocks whose rows keep
+// the key block (the transposed layout).  Per query tile t: S = Q K^T and
+// dP = dO V^T (M = 128 query rows) into TMEM buffer t & 1; the row threads
+// write P and dS = P (dP - D) as bf16 [query][key] tiles into shared memory;
+// then dV^T += dO^T P and dK^T += Q^T dS (M = 128 along d: A is the dO / Q
+// tile read along d, B the P / dS tile read along the keys; for d = 64 the
+// upper 64 rows of M read the neighbouring tile and are never stored) into
+// the item's accumulators (two TMEM pairs, so one item's read-out overlaps
+// the next item's products).  The sums are added into dk and dv (zeroed
+// first), as segments of one column run on several CTAs.  Tiles are
+// numbered across the CTA's items: a tile's Q and dO sit in buffer t & 1
+// until its dV / dK products are done; an item's K and V in buffer (item & 1)
+// until its last S / dP are done.
 template <int BLK, int HD>
 struct DkvShape {
   static constexpr int kQBytes = kTileM * HD * 2;
@@ -566,20 +671,71 @@ struct DkvShape {
   static constexpr int kAtomQ = kTileM * 128;
   static constexpr int kAtomKV = kChunk * 128;
   static constexpr int kPBytes = kTileM * kChunk * 2;      // one [128 queries][64 keys] bf16 tile
-  static constexpr int kOffK = 4 * kQBytes;                // Q, dO of tile t at (t & 1) * 2 * kQBytes
-  static constexpr int kOffV = kOffK + kTile;
-  static constexpr int kOffP = kOffV + kTile;              // P[2], dS[2]
-  static constexpr int kOffBar = kOffP + 4 * kPBytes;
-  // kv_full, q_full[2], s_full[2], pds_full[2], done[2], drain
-  static constexpr int kNumBars = 10;
+  static constexpr int kOffKV = 4 * kQBytes;               // Q, dO of buffer b at b * 2 * kQBytes
+  static constexpr int kOffP = kOffKV + 4 * kTile;         // K, V of buffer b at kOffKV + b * 2 * kTile
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;      // P, dS
+  // kv_full[2] kv_free[2] q_full[2] s_full[2] pds_full done[2] acc_full[2] acc_free[2] drain
+  static constexpr int kBKV = 0, kBKVFree = 2, kBQ = 4, kBS = 6, kBPDS = 8, kBDone = 9, kBAcc = 11,
+                       kBAccFree = 13, kBDrain = 15, kNumBars = 16;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kOffTiles = kOffMisc + 16;          // the segment's query blocks
-  static constexpr int kSmem = kOffTiles + kColumnSegment * 4;
-  static constexpr int kColS = 0, kColDP = 128, kColV = 256, kColK = 320;
+  static constexpr int kSmem = kOffMisc + 16;
+  static constexpr int kColS = 0, kColDP = 128, kColAcc = 256;   // acc pair b: dV at 256 + 128 b, dK 64 further
   static constexpr uint32_t kIdescS = idesc_bf16(kTileM, kChunk, 0, 0);
   static constexpr uint32_t kIdescT = idesc_bf16(kTileM, kChunk, 1, 1);
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
+
+struct DkvItem {
+  int kvh, h0, j, key0, e0, total;
+};
+
+template <int BLK>
+__device__ __forceinline__ bool dkv_item(const Params& p, int x, DkvItem& it) {
+  constexpr int CPB = BLK / kChunk;
+  const int inner = p.n_steps * CPB;
+  const int rank = x / (p.kv_heads * inner);
+  int rem = x - rank * (p.kv_heads * inner);
+  it.kvh = rem / inner;
+  rem -= it.kvh * inner;
+  const int hs = rem / CPB, hh = rem - hs * CPB;
+  it.h0 = it.kvh * p.group + hs * p.pack;
+  const int lh = it.h0 % p.L;
+  const int seg = p.seg_ptr[lh] + rank;
+  if (seg >= p.seg_ptr[lh + 1]) return false;
+  it.j = p.segs[3 * seg];
+  it.e0 = p.segs[3 * seg + 1];
+  it.total = p.segs[3 * seg + 2];
+  it.key0 = it.j * BLK + hh * kChunk;
+  return true;
+}
+
+struct DkvCursor {
+  int x, e, t, y;
+  DkvItem it;
+  bool valid;
+};
+
+template <int BLK>
+__device__ __forceinline__ void dkv_seek(const Params& p, DkvCursor& k) {
+  while (k.x < p.items) {
+    if (dkv_item<BLK>(p, k.x, k.it)) {
+      k.valid = true;
+      return;
+    }
+    k.x += gridDim.x;
+  }
+  k.valid = false;
+}
+
+template <int BLK>
+__device__ __forceinline__ void dkv_advance(const Params& p, DkvCursor& k) {
+  ++k.t;
+  if (++k.e < k.it.total) return;
+  k.e = 0;
+  ++k.y;
+  k.x += gridDim.x;
+  dkv_seek<BLK>(p, k);
+}
 
 template <int BLK, int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -587,55 +743,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                        const Params p) {
   using S = DkvShape<BLK, HD>;
-  constexpr int CPB = BLK / kChunk;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_addr(smem_raw);
   if (base & 1023u) {
     if (threadIdx.x == 0) atomicOr(p.status, kStatusTimeout);
     return;
   }
-  // item -> (segment rank, key/value head, head step, chunk): the longest
-  // segments of every head go first
-  const int inner = p.n_steps * CPB;                     // (head step, chunk) per key/value head
-  const int kv_heads = p.kv_heads;
-  const int rank = blockIdx.x / (kv_heads * inner);
-  int rem = blockIdx.x - rank * (kv_heads * inner);
-  const int kvh = rem / inner;
-  rem -= kvh * inner;
-  const int hs = rem / CPB, hh = rem - hs * CPB;
-  const int h0 = kvh * p.group + hs * p.pack;
-  const int lh = h0 % p.L;
-  const int seg = p.seg_ptr[lh] + rank;
-  if (seg >= p.seg_ptr[lh + 1]) return;                  // this layout head has fewer segments
-  const int j = p.segs[3 * seg], e0 = p.segs[3 * seg + 1], total = p.segs[3 * seg + 2];
-  const int key0 = j * BLK + hh * kChunk;
-
-  auto sQ = [&](int t) { return base + uint32_t(t & 1) * 2 * S::kQBytes; };
-  auto sDO = [&](int t) { return sQ(t) + S::kQBytes; };
-  const uint32_t sK = base + S::kOffK, sV = base + S::kOffV;
-  auto sP = [&](int t) { return base + S::kOffP + uint32_t(t & 1) * S::kPBytes; };
-  auto sDS = [&](int t) { return base + S::kOffP + uint32_t(2 + (t & 1)) * S::kPBytes; };
   const uint32_t bar0 = base + S::kOffBar;
-  const uint32_t bKV = bar0;
-  auto bQ = [&](int t) { return bar0 + 8u * (1 + (t & 1)); };
-  auto bS = [&](int t) { return bar0 + 8u * (3 + (t & 1)); };
-  auto bPDS = [&](int t) { return bar0 + 8u * (5 + (t & 1)); };
-  auto bDone = [&](int t) { return bar0 + 8u * (7 + (t & 1)); };
-  const uint32_t bDrain = bar0 + 8u * 9;
+  auto bar = [&](int idx) { return bar0 + 8u * uint32_t(idx); };
+  auto sQ = [&](int t) { return base + uint32_t(t & 1) * 2 * S::kQBytes; };
+  auto sKV = [&](int y) { return base + S::kOffKV + uint32_t(y & 1) * 2 * S::kTile; };
+  const uint32_t sP = base + S::kOffP, sDS = sP + S::kPBytes;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem_raw + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + S::kOffMisc + 4);
-  int* tiles = reinterpret_cast<int*>(smem_raw + S::kOffTiles);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Ctl ctl{abort_flag, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 9; ++b) mbar_init(bar0 + 8u * b, (b == 5 || b == 6) ? 128u : 1u);
-    mbar_init(bDrain, 1);
+    for (int b = 0; b < S::kNumBars; ++b)
+      mbar_init(bar(b), (b == S::kBPDS || b == S::kBAccFree || b == S::kBAccFree + 1) ? 128u : 1u);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (threadIdx.x < total) tiles[threadIdx.x] = p.row_idx[e0 + threadIdx.x];
-  if (warp == 0) {
+  if (warp == 1) {
     tmem_alloc(base + S::kOffMisc, 512);
     tmem_relinquish();
   }
@@ -645,136 +775,166 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
+    // ---- loads
     if (lane == 0) {
       bool ok = true;
-      int q_loads = 0;
-      auto load_q = [&](int t) {
-        mbar_expect_tx(bQ(t), 2 * S::kQBytes);
-        tma_load_q<BLK, HD>(sQ(t), &tmQ, bQ(t), tiles[t] * BLK, h0);
-        tma_load_q<BLK, HD>(sDO(t), &tmDO, bQ(t), tiles[t] * BLK, h0);
-        ++q_loads;
-      };
-      auto products_s = [&](int t) -> bool {
-        if (!ctl.wait(bQ(t), uint32_t(t >> 1) & 1u)) return false;
-        tc_fence_after();
-        const uint32_t ds = tmem + S::kColS + (t & 1) * kChunk, ddp = tmem + S::kColDP + (t & 1) * kChunk;
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
-          mma_ss(ds, sw128_desc(sQ(t) + ao, 16, 1024), sw128_desc(sK + bo, 16, 1024), S::kIdescS, kk > 0);
-          mma_ss(ddp, sw128_desc(sDO(t) + ao, 16, 1024), sw128_desc(sV + bo, 16, 1024), S::kIdescS, kk > 0);
-        }
-        tc_commit(bS(t));
-        return true;
-      };
-      mbar_expect_tx(bKV, 2 * S::kTile);
-      tma_load_kv<HD>(sK, &tmK, bKV, key0, kvh);
-      tma_load_kv<HD>(sV, &tmV, bKV, key0, kvh);
-      load_q(0);
-      if (total > 1) load_q(1);
-      ok = ctl.wait(bKV, 0);
-      if (ok) ok = products_s(0);
-      if (ok && total > 1) ok = products_s(1);
-      for (int t = 0; t < total && ok; ++t) {
-        // P, dS of tile t are in shared memory, and S, dP of tile t have been read
-        if (!(ok = ctl.wait(bPDS(t), uint32_t(t >> 1) & 1u))) break;
-        tc_fence_after();
-        // dV^T += dO^T P, dK^T += Q^T dS over the tile's 128 query rows
-#pragma unroll
-        for (int kk = 0; kk < kTileM / 16; ++kk) {
-          const uint32_t off = kk * 16 * 128;
-          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-          mma_ss(tmem + S::kColV, sw128_desc(sDO(t) + off, S::kAtomQ, 1024), sw128_desc(sP(t) + off, S::kPBytes, 1024),
-                 S::kIdescT, acc);
-          mma_ss(tmem + S::kColK, sw128_desc(sQ(t) + off, S::kAtomQ, 1024), sw128_desc(sDS(t) + off, S::kPBytes, 1024),
-                 S::kIdescT, acc);
-        }
-        tc_commit(bDone(t));
-        if (t + 2 < total) {
-          // tile t + 2 into buffer t & 1 once tile t's products have read it
-          if (!(ok = ctl.wait(bDone(t), uint32_t(t >> 1) & 1u))) break;
-          load_q(t + 2);
-          if (!(ok = products_s(t + 2))) break;
+      int t = 0, y = 0;
+      DkvItem it;
+      for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
+        if (!dkv_item<BLK>(p, x, it)) continue;
+        if (y >= 2 && !(ok = ctl.wait(bar(S::kBKVFree + (y & 1)), uint32_t((y - 2) >> 1) & 1u))) break;
+        mbar_expect_tx(bar(S::kBKV + (y & 1)), 2 * S::kTile);
+        tma_load_kv<HD>(sKV(y), &tmK, bar(S::kBKV + (y & 1)), it.key0, it.kvh);
+        tma_load_kv<HD>(sKV(y) + S::kTile, &tmV, bar(S::kBKV + (y & 1)), it.key0, it.kvh);
+        ++y;
+        for (int e = 0; e < it.total; ++e, ++t) {
+          if (t >= 2 && !(ok = ctl.wait(bar(S::kBDone + (t & 1)), uint32_t((t - 2) >> 1) & 1u))) break;
+          const int i = p.row_idx[it.e0 + e];
+          mbar_expect_tx(bar(S::kBQ + (t & 1)), 2 * S::kQBytes);
+          tma_load_q<BLK, HD>(sQ(t), &tmQ, bar(S::kBQ + (t & 1)), i * BLK, it.h0);
+          tma_load_q<BLK, HD>(sQ(t) + S::kQBytes, &tmDO, bar(S::kBQ + (t & 1)), i * BLK, it.h0);
         }
       }
-      tc_commit(bDrain);
-      wait_drain(bDrain, 0, kDrainNs);
-      wait_drain(bKV, 0, kDrainNs);
-      for (int t = (q_loads > 2 ? q_loads - 2 : 0); t < q_loads; ++t) wait_drain(bQ(t), uint32_t(t >> 1) & 1u, kDrainNs);
+      if (!ok) {
+        for (int e = (t > 2 ? t - 2 : 0); e < t; ++e) wait_drain(bar(S::kBQ + (e & 1)), uint32_t(e >> 1) & 1u, kDrainNs);
+        for (int e = (y > 2 ? y - 2 : 0); e < y; ++e) wait_drain(bar(S::kBKV + (e & 1)), uint32_t(e >> 1) & 1u, kDrainNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ---- products, issued as their inputs become ready
+    if (lane == 0) {
+      DkvCursor cs{int(blockIdx.x), 0, 0, 0, {}, false}, cd{int(blockIdx.x), 0, 0, 0, {}, false};
+      dkv_seek<BLK>(p, cs);
+      dkv_seek<BLK>(p, cd);
+      uint64_t idle_since = 0;
+      bool ok = true;
+      while (cd.valid && ok) {
+        bool progress = false;
+        // S(t), dP(t): TMEM buffer t & 1 is free once tile t - 2's dV / dK are issued
+        if (cs.valid && cs.t < cd.t + 2 && mbar_test(bar(S::kBKV + (cs.y & 1)), uint32_t(cs.y >> 1) & 1u) &&
+            mbar_test(bar(S::kBQ + (cs.t & 1)), uint32_t(cs.t >> 1) & 1u)) {
+          tc_fence_after();
+          const uint32_t qb = sQ(cs.t), kb = sKV(cs.y), vb = kb + S::kTile;
+          const uint32_t ds = tmem + S::kColS + (cs.t & 1) * kChunk, ddp = tmem + S::kColDP + (cs.t & 1) * kChunk;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
+            mma_ss(ds, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
+            mma_ss(ddp, sw128_desc(qb + S::kQBytes + ao, 16, 1024), sw128_desc(vb + bo, 16, 1024), S::kIdescS,
+                   kk > 0);
+          }
+          tc_commit(bar(S::kBS + (cs.t & 1)));
+          if (cs.e == cs.it.total - 1) tc_commit(bar(S::kBKVFree + (cs.y & 1)));
+          dkv_advance<BLK>(p, cs);
+          progress = true;
+        }
+        // dV^T += dO^T P, dK^T += Q^T dS for tile t, once its P / dS are written
+        if ((cd.t < cs.t || !cs.valid) && mbar_test(bar(S::kBPDS), uint32_t(cd.t) & 1u) &&
+            (cd.e > 0 || cd.y < 2 ||
+             mbar_test(bar(S::kBAccFree + (cd.y & 1)), uint32_t((cd.y - 2) >> 1) & 1u))) {
+          tc_fence_after();
+          const uint32_t qb = sQ(cd.t);
+          const uint32_t accv = tmem + S::kColAcc + uint32_t(cd.y & 1) * 128, acck = accv + 64;
+#pragma unroll
+          for (int kk = 0; kk < kTileM / 16; ++kk) {
+            const uint32_t off = kk * 16 * 128;
+            const uint32_t acc = (cd.e > 0 || kk > 0) ? 1u : 0u;
+            mma_ss(accv, sw128_desc(qb + S::kQBytes + off, S::kAtomQ, 1024), sw128_desc(sP + off, S::kPBytes, 1024),
+                   S::kIdescT, acc);
+            mma_ss(acck, sw128_desc(qb + off, S::kAtomQ, 1024), sw128_desc(sDS + off, S::kPBytes, 1024), S::kIdescT,
+                   acc);
+          }
+          tc_commit(bar(S::kBDone + (cd.t & 1)));
+          if (cd.e == cd.it.total - 1) tc_commit(bar(S::kBAcc + (cd.y & 1)));
+          dkv_advance<BLK>(p, cd);
+          progress = true;
+        }
+        if (progress) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer();
+          if (idle_since == 0) idle_since = now;
+          if (*abort_flag) ok = false;
+          else if (now - idle_since > p.timeout_ns) {
+            *abort_flag = 1;
+            atomicOr(p.status, kStatusTimeout);
+            ok = false;
+          }
+        }
+      }
+      tc_commit(bar(S::kBDrain));
+      wait_drain(bar(S::kBDrain), 0, kDrainNs);
     }
   } else {
+    // ---- rows: P and dS per tile, then each item's dK / dV read-out
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
     const int rl = r - (r / BLK) * BLK;
     bool ok = true;
-    // the row's lse and D for tile t + 1 are fetched while tile t is computed
-    auto row_of = [&](int t, float& lse2, float& dd, bool& live) {
-      int head, tok;
-      const bool real = tile_row<BLK>(p, QTile{tiles[t], h0}, r, head, tok);
-      const size_t rowi = size_t(head) * p.n + (real ? tok : 0);
-      lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
-      dd = real ? p.dsum[rowi] : 0.f;
-      live = real;
-    };
-    float lse2 = 0.f, dd = 0.f;
-    bool live = false;
-    if (total > 0) row_of(0, lse2, dd, live);
-    for (int t = 0; t < total && ok; ++t) {
-      float nlse2 = 0.f, ndd = 0.f;
-      bool nlive = false;
-      if (t + 1 < total) row_of(t + 1, nlse2, ndd, nlive);
-      // causal: in the diagonal block, key (chunk offset + c) > row is dropped
-      const int lim = (tiles[t] == j) ? rl - hh * kChunk : kChunk;
-      ok = __all_sync(0xffffffffu, ctl.wait(bS(t), uint32_t(t >> 1) & 1u));
+    int t = 0, y = 0;
+    DkvItem it;
+    for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
+      if (!dkv_item<BLK>(p, x, it)) continue;
+      const int hh = (it.key0 - it.j * BLK) / kChunk;
+      for (int e = 0; e < it.total; ++e, ++t) {
+        const int i = p.row_idx[it.e0 + e];
+        int head, tok;
+        const bool real = tile_row<BLK>(p, QTile{i, it.h0}, r, head, tok);
+        const size_t rowi = size_t(head) * p.n + (real ? tok : 0);
+        const float lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
+        const float dd = real ? p.dsum[rowi] : 0.f;
+        // causal: in the diagonal block, key (chunk offset + c) > row is dropped
+        const int lim = (i == it.j) ? rl - hh * kChunk : kChunk;
+        ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBS + (t & 1)), uint32_t(t >> 1) & 1u));
+        if (!ok) break;
+        tc_fence_after();
+        float s[kChunk], dp[kChunk], pv[kChunk];
+        const uint32_t cs = lane_base + S::kColS + (t & 1) * kChunk, cdp = lane_base + S::kColDP + (t & 1) * kChunk;
+        tmem_ld32(cs, s);
+        tmem_ld32(cs + 32, s + 32);
+        tmem_ld32(cdp, dp);
+        tmem_ld32(cdp + 32, dp + 32);
+        tmem_wait_ld();
+        p_ds_row(s, dp, pv, p.scale_log2, lse2, dd, lim, real && lse2 > -INFINITY);
+        // the P / dS tiles were last read by tile t - 1's products
+        if (t >= 1) {
+          ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBDone + ((t - 1) & 1)), uint32_t((t - 1) >> 1) & 1u));
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t off = uint32_t(r) * 128 + ((ch ^ (r & 7)) << 4);
+          st_shared_v4(sP + off, pack_bf16(pv[8 * ch], pv[8 * ch + 1]), pack_bf16(pv[8 * ch + 2], pv[8 * ch + 3]),
+                       pack_bf16(pv[8 * ch + 4], pv[8 * ch + 5]), pack_bf16(pv[8 * ch + 6], pv[8 * ch + 7]));
+          st_shared_v4(sDS + off, pack_bf16(s[8 * ch], s[8 * ch + 1]), pack_bf16(s[8 * ch + 2], s[8 * ch + 3]),
+                       pack_bf16(s[8 * ch + 4], s[8 * ch + 5]), pack_bf16(s[8 * ch + 6], s[8 * ch + 7]));
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        mbar_arrive(bar(S::kBPDS));
+      }
+      if (!ok) break;
+      // TMEM lane r holds element d = r of the chunk's 64 key rows
+      ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBAcc + (y & 1)), uint32_t(y >> 1) & 1u));
       if (!ok) break;
       tc_fence_after();
-      float s[kChunk], dp[kChunk], pv[kChunk];
-      const uint32_t cs = lane_base + S::kColS + (t & 1) * kChunk, cd = lane_base + S::kColDP + (t & 1) * kChunk;
-      tmem_ld32(cs, s);
-      tmem_ld32(cs + 32, s + 32);
-      tmem_ld32(cd, dp);
-      tmem_ld32(cd + 32, dp + 32);
-      tmem_wait_ld();
-      p_ds_row(s, dp, pv, p.scale_log2, lse2, dd, lim, live && lse2 > -INFINITY);
-      // buffer t & 1 was last read by tile t - 2's products
-      if (t >= 2) {
-        ok = __all_sync(0xffffffffu, ctl.wait(bDone(t), uint32_t((t - 2) >> 1) & 1u));
-        if (!ok) break;
-      }
-      // row r of the [query][key] tiles, 128-byte swizzled
-      const uint32_t tp = sP(t), td = sDS(t);
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t off = uint32_t(r) * 128 + ((ch ^ (r & 7)) << 4);
-        st_shared_v4(tp + off, pack_bf16(pv[8 * ch], pv[8 * ch + 1]), pack_bf16(pv[8 * ch + 2], pv[8 * ch + 3]),
-                     pack_bf16(pv[8 * ch + 4], pv[8 * ch + 5]), pack_bf16(pv[8 * ch + 6], pv[8 * ch + 7]));
-        st_shared_v4(td + off, pack_bf16(s[8 * ch], s[8 * ch + 1]), pack_bf16(s[8 * ch + 2], s[8 * ch + 3]),
-                     pack_bf16(s[8 * ch + 4], s[8 * ch + 5]), pack_bf16(s[8 * ch + 6], s[8 * ch + 7]));
-      }
-      fence_proxy_async();
-      tc_fence_before();
-      mbar_arrive(bPDS(t));
-      lse2 = nlse2;
-      dd = ndd;
-      live = nlive;
-    }
-    // TMEM lane r holds element d = r of the chunk's 64 key rows
-    if (ok && total > 0) ok = __all_sync(0xffffffffu, ctl.wait(bDone(total - 1), uint32_t((total - 1) >> 1) & 1u));
-    if (ok && total > 0) {
-      tc_fence_after();
       float vk[kChunk], vv[kChunk];
-      tmem_ld32(lane_base + S::kColK, vk);
-      tmem_ld32(lane_base + S::kColK + 32, vk + 32);
-      tmem_ld32(lane_base + S::kColV, vv);
-      tmem_ld32(lane_base + S::kColV + 32, vv + 32);
+      const uint32_t accv = lane_base + S::kColAcc + uint32_t(y & 1) * 128;
+      tmem_ld32(accv + 64, vk);
+      tmem_ld32(accv + 96, vk + 32);
+      tmem_ld32(accv, vv);
+      tmem_ld32(accv + 32, vv + 32);
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(S::kBAccFree + (y & 1)));
+      ++y;
       if (r < HD) {
 #pragma unroll
         for (int c = 0; c < kChunk; ++c) {
-          const int key = key0 + c;
+          const int key = it.key0 + c;
           if (key < p.n) {
-            const size_t at = (size_t(kvh) * p.n + key) * HD + r;
+            const size_t at = (size_t(it.kvh) * p.n + key) * HD + r;
             atomicAdd(p.dk + at, vk[c] * p.scale);
             atomicAdd(p.dv + at, vv[c]);
           }
@@ -784,7 +944,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -868,7 +1028,7 @@ int encode_q(CUtensorMap* m, const void* ptr, int heads, int n, int d, int blk) 
 
 struct Launch {
   const void *q, *k, *v, *o, *dout;
-  int heads, kv_heads, n, items_dq, items_dkv;
+  int heads, kv_heads, n, items_dq, items_dkv, sms;
   size_t dq_rows;
   float* dsum;
   cudaStream_t stream;
@@ -924,8 +1084,12 @@ int launch_instance(const Launch& a, const bwd::Params& p) {
   const unsigned rows_grid = unsigned((a.dq_rows + 7) / 8);
   bwd::bsa_bwd_rowdot_kernel<HD><<<rows_grid, 256, 0, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.dsum, a.dq_rows);
-  if (a.items_dq > 0) kq<<<a.items_dq, bwd::kThreads, smem_q, a.stream>>>(mq, mdo, mk, mv, p);
-  if (a.items_dkv > 0) kkv<<<a.items_dkv, bwd::kThreads, smem_kv, a.stream>>>(mq, mdo, mk, mv, p);
+  bwd::Params pq = p, pk = p;
+  pq.items = a.items_dq;
+  pk.items = a.items_dkv;
+  if (a.items_dq > 0) kq<<<a.items_dq < a.sms ? a.items_dq : a.sms, bwd::kThreads, smem_q, a.stream>>>(mq, mdo, mk, mv, pq);
+  if (a.items_dkv > 0)
+    kkv<<<a.items_dkv < a.sms ? a.items_dkv : a.sms, bwd::kThreads, smem_kv, a.stream>>>(mq, mdo, mk, mv, pk);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
   return BSA_OK;
@@ -985,6 +1149,7 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   p.n = n;
   p.nb = layout->nb;
   p.L = layout->L;
+  p.heads = heads;
   p.kv_heads = kv_heads;
   p.group = group;
   p.pack = pack;
@@ -992,7 +1157,10 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   p.scale = scale;
   p.scale_log2 = float(double(scale) * 1.4426950408889634);
   p.timeout_ns = 1000000000ull;   // 1 s: never reached in a correct run
-  Launch a{q, k, v, o, dout, heads, kv_heads, n, int(items_dq), int(items_dkv), size_t(heads) * n, workspace,
+  int sms = 0;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, cur);
+  if (e != cudaSuccess || sms < 1) return set_error(BSA_ERR_CUDA, "cannot query the SM count");
+  Launch a{q, k, v, o, dout, heads, kv_heads, n, int(items_dq), int(items_dkv), sms, size_t(heads) * n, workspace,
            static_cast<cudaStream_t>(stream)};
   if (B == 64 && d == 128) return launch_instance<64, 128>(a, p);
   if (B == 64 && d == 64) return launch_instance<64, 64>(a, p);
