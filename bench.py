@@ -466,6 +466,8 @@ def main():
     backward = ({name: bench_backward(WORKLOADS[name], dev, stream, flush, bsa, torch)
                  for name in (HEADLINE, "band_global_32k")}
                 if rank == 0 and not args.no_per_config else None)
+    bsbr = bench_bsbr(WORKLOADS["bsbr_block_diagonal"], dev, stream, flush, bsa, torch) \
+        if rank == 0 and not args.no_per_config else None
 
     peaks, peak_src = load_peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -511,6 +513,7 @@ def main():
             "per_config": per_config,
             "decode": decode,
             "backward": backward,
+            "bsbr": bsbr,
         }
         print(json.dumps(line), flush=True)
     sampler.stop()
@@ -598,6 +601,58 @@ def bench_backward(w, dev, stream, flush, bsa, torch, steps=10, warmup=3):
     return {"ms_median": med, "effective_tflops": tf, "frac_of_measured_peak": tf / peak,
             "algorithmic_flops": flops, "kept_pairs": pairs, "launches_per_call": 3,
             "data": "torch.randn on device, seed 4321; L2 flushed between steps"}
+
+
+def bench_bsbr(w, dev, stream, flush, bsa, torch, steps=20, warmup=3):
+    """BSBR attention on its workload: the within-chunk forward (bsa_forward on
+    the block-diagonal layout) plus the between-chunk retrieval
+    (bsa_bsbr_retrieval), and the retrieval alone.  The retrieval's
+    algorithmic HBM bytes: k and v read, the chunk states and meta keys
+    written and read once, q read, o read and written."""
+    lay = bsa.Layout.for_workload(w, dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(777)
+    q = torch.randn((w.heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    k = torch.randn((w.kv_heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    v = torch.randn((w.kv_heads, w.n, w.d), device=dev, generator=gen).to(torch.bfloat16)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.heads, w.n), dtype=torch.float32, device=dev)
+    need = bsa.bsa_bsbr_workspace_bytes(w.n, w.B, w.kv_heads, w.d)
+    ws = torch.empty(((need + 15) // 16) * 4, dtype=torch.float32, device=dev)
+    scale = 1.0 / math.sqrt(w.d)
+    chunks = -(-w.n // w.B)
+    res = {}
+    for leg in ("forward_plus_retrieval", "retrieval_only"):
+        ev = []
+        for st in range(warmup + steps):
+            flush.fill_(float(st))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            if leg == "forward_plus_retrieval":
+                bsa.bsa_forward(q, k, v, lay.handle, w.B, w.n, w.heads, w.kv_heads, w.d, scale, o, lse, stream)
+            bsa.bsa_bsbr_retrieval(q, k, v, lay.handle, w.B, w.n, w.heads, w.kv_heads, w.d, scale, o, ws,
+                                   ws.numel() * 4, stream)
+            b.record(stream)
+            if st >= warmup:
+                ev.append((a, b))
+        torch.cuda.synchronize()
+        bsa.bsa_get_status(lay.handle)
+        ts = sorted(a.elapsed_time(b) for a, b in ev)
+        res[leg] = {"us_median": ts[len(ts) // 2] * 1e3}
+    elem = w.n * w.d * 2
+    bytes_ret = (2 * w.kv_heads * elem + 3 * w.heads * elem
+                 + 2 * w.kv_heads * chunks * w.d * (w.d + 1) * 4)
+    us = res["retrieval_only"]["us_median"]
+    hbm = float(load_peaks()[0].get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = bytes_ret / (us * 1e-6) / 1e9
+    res["retrieval_only"].update({"algorithmic_bytes": bytes_ret, "gbs": gbs, "frac_of_measured_hbm": gbs / hbm,
+                                  "launches": 2})
+    res["workload"] = (f"BSBR: batch {w.batch} x {w.q_heads} heads, n={w.n}, d={w.d}, chunks of B={w.B} "
+                       f"({chunks} chunks)")
+    res["data"] = "torch.randn on device, seed 777; L2 flushed between steps"
+    lay.close()
+    del q, k, v, o, lse, ws
+    return res
 
 
 def bench_decode(dev, stream, flush, bsa, torch, batches=(1, 32), steps=20, warmup=3):

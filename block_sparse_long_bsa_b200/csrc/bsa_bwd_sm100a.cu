@@ -10,15 +10,19 @@
 //   dv_u = sum_t P_tu dO_t.
 // P is rebuilt from the forward's lse, so no n x n matrix is stored.
 //
-// Three launches on the caller's stream: D (one warp per row), then the dq
-// kernel (query tiles, each walking its CSR row of kept blocks) and the dk/dv
-// kernel (segments of a key block's column of the transposed layout, each
-// walking the query tiles that read it).  Both product kernels are
-// persistent, one CTA per SM, 192 threads: warp 0 issues the TMA loads; one
+// Launches on the caller's stream: a clear of the dk / dv rows that are
+// summed by several CTAs (or of all of dk, dv), D (one warp per row), then the
+// dq kernel (query tiles, each walking its CSR row of kept blocks) and the
+// dk/dv kernel (segments of a key block's column of the transposed layout,
+// each walking the query tiles that read it).  Both product kernels are
+// persistent, one CTA per SM, 320 threads: warp 0 decodes the CTA's work
+// items into a ring of shared-memory slots and issues the TMA loads; one
 // thread of warp 1 issues the tcgen05 products, each as soon as its inputs
 // are ready (two kinds of product interleave, so neither waits behind the
-// other); warps 2-5 hold one tile row per thread (warp w reaches TMEM lanes
-// 32 (w % 4) ..) and rebuild P and dS.  Every product is a
+// other; the thread polls with non-blocking barrier tests, which reacts
+// faster than suspending waits); warps 2-9 rebuild P and dS, two threads per
+// tile row (warp w reaches TMEM lanes 32 (w % 4) ..; warps 2-5 take the first
+// 32 keys of each 64-key chunk, warps 6-9 the other 32).  Every product is a
 // 128-row bf16 x bf16 -> fp32 tcgen05 MMA accumulating in TMEM.  Every
 // mbarrier wait is bounded: one that runs out sets the layout's status word,
 // the CTA drains what it has in flight, releases TMEM and returns.
@@ -256,9 +260,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo_bytes
 }
 
 // ---------------------------------------------------------------- shared
-constexpr int kThreads = 192;        // warp 0: loads; warp 1: products; warps 2-5: one tile row per thread
+constexpr int kThreads = 320;        // warp 0: item ring and loads; warp 1: products; warps 2-9: rows
+constexpr int kRowThreads = 256;     // two threads per tile row, one per half of a 64-key chunk
+constexpr int kRowWarps = 8;
 constexpr int kTileM = 128;          // rows of every product tile (tcgen05 M = 128)
 constexpr int kChunk = 64;           // keys per chunk
+constexpr int kHalf = 32;            // keys per row thread
+constexpr int kRing = 8;             // decoded work items in flight
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint64_t kDrainNs = 200000000ull;
 
@@ -273,6 +281,7 @@ struct Params {
   const int32_t* row_ptr;
   const int32_t* col_idx;
   const int32_t* order;
+  const int32_t* col_ptr;
   const int32_t* row_idx;
   const int32_t* seg_ptr;
   const int32_t* segs;
@@ -304,20 +313,56 @@ __device__ __forceinline__ bool tile_row(const Params& p, const QTile& t, int r,
   return sub < p.pack && tok < p.n;
 }
 
-// P and dS of one tile row against one 64-key chunk, from the raw scores s
-// (q.k) and dP (dO.v): P = exp(scale s - lse), dS = P (dP - D).  Keys past
-// `lim` (causal, diagonal block) and rows that are not real get 0.  dS
-// overwrites s.
-__device__ __forceinline__ void p_ds_row(float* s, const float* dp, float* pv, float sl2, float lse2, float dd,
-                                         int lim, bool live) {
+// P and dS of one row against 32 keys of a chunk, from the raw scores s (q.k)
+// and dP (dO.v): P = exp(scale s - lse), dS = P (dP - D).  Keys past `lim`
+// (causal, diagonal block) and rows that are not live get 0.  dS overwrites s.
+__device__ __forceinline__ void p_ds_half(float* s, const float* dp, float* pv, float sl2, float lse2, float dd,
+                                          int lim, bool live) {
 #pragma unroll
-  for (int c = 0; c < kChunk; ++c) {
+  for (int c = 0; c < kHalf; ++c) {
     const bool keep = live && c <= lim;
     const float pr = keep ? ex2(fmaf(s[c], sl2, -lse2)) : 0.f;
     pv[c] = pr;
     s[c] = pr * (dp[c] - dd);
   }
 }
+
+// Row-thread coordinates: warps 2-9, warp w reaching TMEM lanes 32 (w % 4);
+// warps 2-5 take keys 0-31 of each chunk, warps 6-9 keys 32-63.
+struct RowRole {
+  int r, hf;
+  uint32_t lane_base;
+};
+__device__ __forceinline__ RowRole row_role(uint32_t tmem) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q4 = warp & 3;
+  RowRole rr;
+  rr.r = q4 * 32 + lane;
+  rr.hf = (warp - 2) >> 2;
+  rr.lane_base = tmem + (uint32_t(q4 * 32) << 16);
+  return rr;
+}
+
+// Bounded polling of several conditions by one thread: true while it may go
+// on; after `timeout_ns` without progress it raises the abort flag.
+struct Idle {
+  uint64_t since = 0;
+  __device__ __forceinline__ bool step(bool progress, const Ctl& ctl) {
+    if (progress) {
+      since = 0;
+      return true;
+    }
+    if (*ctl.abort) return false;
+    const uint64_t now = globaltimer();
+    if (since == 0) since = now;
+    if (now - since > ctl.timeout_ns) {
+      *ctl.abort = 1;
+      atomicOr(ctl.status, kStatusTimeout);
+      return false;
+    }
+    return true;
+  }
+};
 
 // ---------------------------------------------------------------- D = rowsum(dO * o)
 // One warp per query row: D_t = sum_u P_tu dP_tu, which equals <dO_t, o_t>.
@@ -343,16 +388,39 @@ __global__ void __launch_bounds__(256) bsa_bwd_rowdot_kernel(const __nv_bfloat16
   if (lane == 0) dsum[row] = acc;
 }
 
+// ---------------------------------------------------------------- dk, dv clear
+// Zeroes the dk and dv rows of key blocks that do not get exactly one
+// store: blocks no query reads (no segment) and blocks whose column is cut
+// into several segments (their sums are added by several CTAs).  Used when
+// each key/value head has one head step; otherwise all of dk, dv are cleared.
+template <int HD>
+__global__ void __launch_bounds__(256) bsa_bwd_clear_kernel(const Params p, int B) {
+  const int kvh = blockIdx.x / p.nb, j = blockIdx.x - kvh * p.nb;
+  const int lh = (kvh * p.group) % p.L;
+  const int len = p.col_ptr[size_t(lh) * p.nb + j + 1] - p.col_ptr[size_t(lh) * p.nb + j];
+  if (len >= 1 && len <= kColumnSegment) return;
+  const int t0 = j * B, t1 = min(p.n, t0 + B);
+  float4* dk = reinterpret_cast<float4*>(p.dk + (size_t(kvh) * p.n + t0) * HD);
+  float4* dv = reinterpret_cast<float4*>(p.dv + (size_t(kvh) * p.n + t0) * HD);
+  const int count = (t1 - t0) * HD / 4;
+  for (int e = threadIdx.x; e < count; e += blockDim.x) {
+    dk[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    dv[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
 // ---------------------------------------------------------------- dQ
-// Persistent: one CTA per SM walks query tiles (longest row first, every
-// gridDim-th).  Per 64-key chunk c of a tile's kept blocks: S = Q K_c^T and
-// dP = dO V_c^T into TMEM buffer c & 1; the row threads turn them into
-// dS = P (dP - D), rounded to bf16 over the S buffer; then dQ += dS K_c
-// (A = dS read from TMEM, B = K_c read along d) into the tile's accumulator
-// (two TMEM accumulators, so one tile's read-out overlaps the next tile's
-// products).  Chunks are numbered across the CTA's tiles: K_c sits in slot
-// c % 4 until dQ_c is done, V_c in slot c % 2 until S_c / dP_c are done, and
-// a tile's Q and dO in buffer (tile & 1) until its last S / dP are done.
+// Persistent: one CTA per SM walks query tiles (head group by head group,
+// longest row first inside one, every gridDim-th).  Warp 0 decodes each tile into a ring of shared-memory slots
+// (read by the other warps) and loads its Q, dO, K and V tiles.  Per 64-key
+// chunk c of a tile's kept blocks: S = Q K_c^T and dP = dO V_c^T into TMEM
+// buffer c & 1; the row threads turn them into dS = P (dP - D), rounded to
+// bf16 and packed over their own S columns; then dQ += dS K_c (A = dS read
+// from TMEM, B = K_c read along d) into the tile's accumulator (two TMEM
+// accumulators, so one tile's read-out overlaps the next tile's products).
+// Chunks are numbered across the CTA's tiles: K_c sits in slot c % 4 until
+// dQ_c is done, V_c in slot c % 2 until S_c / dP_c are done, and a tile's Q
+// and dO in buffer (tile & 1) until its last S / dP are done.
 template <int BLK, int HD>
 struct DqShape {
   static constexpr int kCPB = BLK / kChunk;
@@ -364,10 +432,11 @@ struct DqShape {
   static constexpr int kOffK = 4 * kQBytes;                // Q, dO of buffer b at b * 2 * kQBytes
   static constexpr int kOffV = kOffK + kRingK * kTile;
   static constexpr int kOffBar = kOffV + kRingV * kTile;
-  // q_full[2] q_free[2] k_full[4] k_free[4] v_full[2] s_full[2] ds_full[2] acc_full[2] acc_free[2] drain
   static constexpr int kBQ = 0, kBQFree = 2, kBK = 4, kBKFree = 8, kBV = 12, kBS = 14, kBDS = 16, kBAcc = 18,
-                       kBAccFree = 20, kBDrain = 22, kNumBars = 23;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+                       kBAccFree = 20, kBItem = 22, kBItemFree = 22 + kRing, kBDrain = 22 + 2 * kRing,
+                       kNumBars = 23 + 2 * kRing;
+  static constexpr int kOffRing = ((kOffBar + kNumBars * 8 + 15) / 16) * 16;
+  static constexpr int kOffMisc = kOffRing + kRing * 32;
   static constexpr int kSmem = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColQ = 256;
   static constexpr uint32_t kIdescS = idesc_bf16(kTileM, kChunk, 0, 0);
@@ -376,61 +445,59 @@ struct DqShape {
   static_assert(kColQ + 2 * HD <= 512, "TMEM columns");
 };
 
-struct DqItem {
-  QTile tile;
-  int kvh, start, nch, diag_first;
+// One decoded query tile (a ring slot).  last = 1 marks the end of the CTA's list.
+struct DqSlot {
+  int i, h0, kvh, start, nch, diag_first, last, pad;
 };
 
 template <int BLK>
-__device__ __forceinline__ DqItem dq_item(const Params& p, int x) {
+__device__ __forceinline__ DqSlot dq_decode(const Params& p, int x) {
   constexpr int CPB = BLK / kChunk;
-  const int n_hg = p.heads / p.pack;
-  const int rank = x / n_hg, hg = x - rank * n_hg;
-  DqItem it;
-  it.tile.h0 = hg * p.pack;
-  const int lh = it.tile.h0 % p.L;
-  it.tile.i = p.order[size_t(lh) * p.nb + rank];
-  it.kvh = it.tile.h0 / p.group;
-  const size_t lrow = size_t(lh) * p.nb + it.tile.i;
-  it.start = p.row_ptr[lrow];
-  const int len = p.row_ptr[lrow + 1] - it.start;
-  it.nch = len * CPB;
-  const bool diag_last = len > 0 && p.col_idx[it.start + len - 1] == it.tile.i;
-  it.diag_first = diag_last ? it.nch - CPB : it.nch;
-  return it;
+  DqSlot s;
+  s.pad = 0;
+  if (x >= p.items) {
+    s.last = 1;
+    s.i = s.h0 = s.kvh = s.start = s.nch = s.diag_first = 0;
+    return s;
+  }
+  s.last = 0;
+  // head group by head group (the K / V working set in flight is about one
+  // key/value head and stays in L2), longest row first inside a head group
+  const int hg = x / p.nb, rank = x - hg * p.nb;
+  s.h0 = hg * p.pack;
+  const int lh = s.h0 % p.L;
+  s.i = p.order[size_t(lh) * p.nb + rank];
+  s.kvh = s.h0 / p.group;
+  const size_t lrow = size_t(lh) * p.nb + s.i;
+  s.start = p.row_ptr[lrow];
+  const int len = p.row_ptr[lrow + 1] - s.start;
+  s.nch = len * CPB;
+  const bool diag_last = len > 0 && p.col_idx[s.start + len - 1] == s.i;
+  s.diag_first = diag_last ? s.nch - CPB : s.nch;
+  return s;
 }
 
-// A position in a CTA's stream of chunks: item x (global index), chunk c of
-// it, global chunk number g, and the count of non-empty items before it.
+__device__ __forceinline__ DqSlot read_slot(const uint8_t* ring, int k) {
+  const volatile int* v = reinterpret_cast<const volatile int*>(ring + (k % kRing) * 32);
+  DqSlot s;
+  s.i = v[0];
+  s.h0 = v[1];
+  s.kvh = v[2];
+  s.start = v[3];
+  s.nch = v[4];
+  s.diag_first = v[5];
+  s.last = v[6];
+  s.pad = 0;
+  return s;
+}
+
+// A position in a CTA's stream of chunks: ring item k, chunk c of it, global
+// chunk number g, and the count of non-empty items before it.
 struct DqCursor {
-  int x, c, g, xi;
-  DqItem it;
+  int k, c, g, xi;
+  DqSlot it;
   bool valid;
 };
-
-template <int BLK>
-__device__ __forceinline__ void dq_seek(const Params& p, DqCursor& k) {
-  // skip empty items from k.x on
-  while (k.x < p.items) {
-    k.it = dq_item<BLK>(p, k.x);
-    if (k.it.nch > 0) {
-      k.valid = true;
-      return;
-    }
-    k.x += gridDim.x;
-  }
-  k.valid = false;
-}
-
-template <int BLK>
-__device__ __forceinline__ void dq_advance(const Params& p, DqCursor& k) {
-  ++k.g;
-  if (++k.c < k.it.nch) return;
-  k.c = 0;
-  ++k.xi;
-  k.x += gridDim.x;
-  dq_seek<BLK>(p, k);
-}
 
 template <int BLK, int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -450,14 +517,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sQ = [&](int b) { return base + uint32_t(b) * 2 * S::kQBytes; };
   auto sK = [&](int g) { return base + S::kOffK + uint32_t(g % S::kRingK) * S::kTile; };
   auto sV = [&](int g) { return base + S::kOffV + uint32_t(g % S::kRingV) * S::kTile; };
+  uint8_t* ring = smem_raw + S::kOffRing;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem_raw + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + S::kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Ctl ctl{abort_flag, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < S::kNumBars; ++b)
-      mbar_init(bar(b), (b == S::kBDS || b == S::kBDS + 1 || b == S::kBAccFree || b == S::kBAccFree + 1) ? 128u : 1u);
+    for (int b = 0; b < S::kNumBars; ++b) {
+      uint32_t count = 1;
+      if (b == S::kBDS || b == S::kBDS + 1 || b == S::kBAccFree || b == S::kBAccFree + 1) count = kRowThreads;
+      if (b >= S::kBItemFree && b < S::kBItemFree + kRing) count = kRowWarps + 1;
+      mbar_init(bar(b), count);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -471,25 +543,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
-    // ---- loads
+    // ---- item ring and loads
     if (lane == 0) {
       bool ok = true;
       int nk = 0, nv = 0, xi = 0;   // K, V and Q / dO loads issued (chunk g's K is load g)
-      for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
-        const DqItem it = dq_item<BLK>(p, x);
+      for (int k = 0, x = blockIdx.x; ok; ++k, x += gridDim.x) {
+        if (k >= kRing && !(ok = ctl.wait(bar(S::kBItemFree + k % kRing), uint32_t((k - kRing) / kRing) & 1u))) break;
+        const DqSlot it = dq_decode<BLK>(p, x);
+        volatile int* v = reinterpret_cast<volatile int*>(ring + (k % kRing) * 32);
+        v[0] = it.i;
+        v[1] = it.h0;
+        v[2] = it.kvh;
+        v[3] = it.start;
+        v[4] = it.nch;
+        v[5] = it.diag_first;
+        v[6] = it.last;
+        mbar_arrive(bar(S::kBItem + k % kRing));
+        if (it.last) break;
         if (it.nch == 0) continue;
         const int b = xi & 1;
         if (xi >= 2 && !(ok = ctl.wait(bar(S::kBQFree + b), uint32_t((xi - 2) >> 1) & 1u))) break;
         mbar_expect_tx(bar(S::kBQ + b), 2 * S::kQBytes);
-        tma_load_q<BLK, HD>(sQ(b), &tmQ, bar(S::kBQ + b), it.tile.i * BLK, it.tile.h0);
-        tma_load_q<BLK, HD>(sQ(b) + S::kQBytes, &tmDO, bar(S::kBQ + b), it.tile.i * BLK, it.tile.h0);
+        tma_load_q<BLK, HD>(sQ(b), &tmQ, bar(S::kBQ + b), it.i * BLK, it.h0);
+        tma_load_q<BLK, HD>(sQ(b) + S::kQBytes, &tmDO, bar(S::kBQ + b), it.i * BLK, it.h0);
         ++xi;
         for (int c = 0; c < it.nch; ++c) {
           const int g = nk;
           const int key0 = p.col_idx[it.start + c / CPB] * BLK + (c % CPB) * kChunk;
           // K slot g % 4 held chunk g - 4 until its dQ product; V slot g % 2
           // held chunk g - 2 until its S / dP products
-          if (g >= S::kRingK && !(ok = ctl.wait(bar(S::kBKFree + g % S::kRingK), uint32_t((g - S::kRingK) / S::kRingK) & 1u)))
+          if (g >= S::kRingK &&
+              !(ok = ctl.wait(bar(S::kBKFree + g % S::kRingK), uint32_t((g - S::kRingK) / S::kRingK) & 1u)))
             break;
           mbar_expect_tx(bar(S::kBK + g % S::kRingK), S::kTile);
           tma_load_kv<HD>(sK(g), &tmK, bar(S::kBK + g % S::kRingK), key0, it.kvh);
@@ -512,11 +596,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---- products, issued as their inputs become ready
     if (lane == 0) {
-      DqCursor cs{int(blockIdx.x), 0, 0, 0, {}, false}, cd{int(blockIdx.x), 0, 0, 0, {}, false};
-      dq_seek<BLK>(p, cs);
-      dq_seek<BLK>(p, cd);
-      uint64_t idle_since = 0;
       bool ok = true;
+      // cursor load: the next non-empty item from ring item k on; the dQ
+      // cursor, the later of the two, hands each slot back once copied
+      auto seek = [&](DqCursor& cu, bool release) {
+        while (ok) {
+          if (!(ok = ctl.wait(bar(S::kBItem + cu.k % kRing), uint32_t(cu.k / kRing) & 1u))) break;
+          cu.it = read_slot(ring, cu.k);
+          if (release) mbar_arrive(bar(S::kBItemFree + cu.k % kRing));
+          if (cu.it.last) {
+            cu.valid = false;
+            return;
+          }
+          if (cu.it.nch > 0) {
+            cu.valid = true;
+            return;
+          }
+          ++cu.k;
+        }
+        cu.valid = false;
+      };
+      auto advance = [&](DqCursor& cu, bool release) {
+        ++cu.g;
+        if (++cu.c < cu.it.nch) return;
+        cu.c = 0;
+        ++cu.xi;
+        ++cu.k;
+        seek(cu, release);
+      };
+      DqCursor cs{0, 0, 0, 0, {}, false}, cd{0, 0, 0, 0, {}, false};
+      seek(cs, false);
+      seek(cd, true);
+      Idle idle;
       while (cd.valid && ok) {
         bool progress = false;
         if (cs.valid && cs.g < cd.g + 2 && mbar_test(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u) &&
@@ -534,110 +645,117 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(S::kBS + (cs.g & 1)));
           if (cs.c == cs.it.nch - 1) tc_commit(bar(S::kBQFree + (cs.xi & 1)));
-          dq_advance<BLK>(p, cs);
+          advance(cs, false);
           progress = true;
         }
-        if (cd.g < cs.g || !cs.valid) {
-          if (mbar_test(bar(S::kBDS + (cd.g & 1)), uint32_t(cd.g >> 1) & 1u) &&
-              (cd.c > 0 || cd.xi < 2 ||
-               mbar_test(bar(S::kBAccFree + (cd.xi & 1)), uint32_t((cd.xi - 2) >> 1) & 1u))) {
-            tc_fence_after();
-            const uint32_t pa = tmem + S::kColS + (cd.g & 1) * kChunk, kb = sK(cd.g);
-            const uint32_t acc = tmem + S::kColQ + uint32_t(cd.xi & 1) * HD;
+        if ((cd.g < cs.g || !cs.valid) && mbar_test(bar(S::kBDS + (cd.g & 1)), uint32_t(cd.g >> 1) & 1u) &&
+            (cd.c > 0 || cd.xi < 2 ||
+             mbar_test(bar(S::kBAccFree + (cd.xi & 1)), uint32_t((cd.xi - 2) >> 1) & 1u))) {
+          tc_fence_after();
+          // dS of keys 0-31 is packed at columns 0-15 of the S buffer, keys 32-63 at 32-47
+          const uint32_t pa = tmem + S::kColS + (cd.g & 1) * kChunk, kb = sK(cd.g);
+          const uint32_t acc = tmem + S::kColQ + uint32_t(cd.xi & 1) * HD;
 #pragma unroll
-            for (int kk = 0; kk < kChunk / 16; ++kk)
-              mma_ts(acc, pa + kk * 8, sw128_desc(kb + kk * 16 * 128, S::kAtomKV, 1024), S::kIdescDQ,
-                     (cd.c > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(bar(S::kBKFree + cd.g % S::kRingK));
-            if (cd.c == cd.it.nch - 1) tc_commit(bar(S::kBAcc + (cd.xi & 1)));
-            dq_advance<BLK>(p, cd);
-            progress = true;
-          }
+          for (int kk = 0; kk < kChunk / 16; ++kk)
+            mma_ts(acc, pa + (kk >> 1) * 32 + (kk & 1) * 8, sw128_desc(kb + kk * 16 * 128, S::kAtomKV, 1024),
+                   S::kIdescDQ, (cd.c > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(S::kBKFree + cd.g % S::kRingK));
+          if (cd.c == cd.it.nch - 1) tc_commit(bar(S::kBAcc + (cd.xi & 1)));
+          advance(cd, true);
+          progress = true;
         }
-        if (progress) {
-          idle_since = 0;
-        } else {
-          const uint64_t now = globaltimer();
-          if (idle_since == 0) idle_since = now;
-          if (*abort_flag) ok = false;
-          else if (now - idle_since > p.timeout_ns) {
-            *abort_flag = 1;
-            atomicOr(p.status, kStatusTimeout);
-            ok = false;
-          }
-        }
+        ok = ok && idle.step(progress, ctl);
       }
       tc_commit(bar(S::kBDrain));
       wait_drain(bar(S::kBDrain), 0, kDrainNs);
     }
   } else {
-    // ---- rows: dS, then each tile's dQ read-out
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
-    const int rl = r - (r / BLK) * BLK;
+    // ---- rows: dS, then each tile's dQ read-out (half of the columns per thread)
+    const RowRole rr = row_role(tmem);
+    const int rl = rr.r - (rr.r / BLK) * BLK;
+    constexpr int kCols = HD / 2;
     bool ok = true;
     int g = 0, xi = 0;
-    for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
-      const DqItem it = dq_item<BLK>(p, x);
+    // the row's lse and D of the next item are fetched while the current one ends
+    float nlse2 = 0.f, ndd = 0.f;
+    bool have_next = false;
+    for (int k = 0; ok; ++k) {
+      ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBItem + k % kRing), uint32_t(k / kRing) & 1u));
+      if (!ok) break;
+      const DqSlot it = read_slot(ring, k);
+      if (it.last) break;
       int head, tok;
-      const bool real = tile_row<BLK>(p, it.tile, r, head, tok);
+      const bool real = tile_row<BLK>(p, QTile{it.i, it.h0}, rr.r, head, tok);
       const size_t rowi = size_t(head) * p.n + (real ? tok : 0);
-      float* out = p.dq + rowi * HD;
+      float* out = p.dq + rowi * HD + rr.hf * kCols;
+      float lse2, dd;
+      if (have_next) {
+        lse2 = nlse2;
+        dd = ndd;
+      } else {
+        lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
+        dd = real ? p.dsum[rowi] : 0.f;
+      }
+      have_next = false;
       if (it.nch == 0) {
         if (real) {
 #pragma unroll
-          for (int e = 0; e < HD; e += 4) *reinterpret_cast<float4*>(out + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int e = 0; e < kCols; e += 4) *reinterpret_cast<float4*>(out + e) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        continue;
-      }
-      const float lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
-      const float dd = real ? p.dsum[rowi] : 0.f;
-      const bool live = real && lse2 > -INFINITY;
-      for (int c = 0; c < it.nch; ++c, ++g) {
-        ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBS + (g & 1)), uint32_t(g >> 1) & 1u));
-        if (!ok) break;
-        tc_fence_after();
-        float s[kChunk], dp[kChunk], pv[kChunk];
-        const uint32_t cs = lane_base + S::kColS + (g & 1) * kChunk, cdp = lane_base + S::kColDP + (g & 1) * kChunk;
-        tmem_ld32(cs, s);
-        tmem_ld32(cs + 32, s + 32);
-        tmem_ld32(cdp, dp);
-        tmem_ld32(cdp + 32, dp + 32);
-        tmem_wait_ld();
-        const int lim = c >= it.diag_first ? rl - (c - it.diag_first) * kChunk : kChunk;
-        p_ds_row(s, dp, pv, p.scale_log2, lse2, dd, lim, live);
-#pragma unroll
-        for (int h = 0; h < kChunk / 32; ++h) {
+      } else {
+        const bool live = real && lse2 > -INFINITY;
+        for (int c = 0; c < it.nch; ++c, ++g) {
+          ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBS + (g & 1)), uint32_t(g >> 1) & 1u));
+          if (!ok) break;
+          tc_fence_after();
+          float s[kHalf], dp[kHalf], pv[kHalf];
+          const uint32_t cs = rr.lane_base + S::kColS + (g & 1) * kChunk + rr.hf * kHalf;
+          tmem_ld32(cs, s);
+          tmem_ld32(rr.lane_base + S::kColDP + (g & 1) * kChunk + rr.hf * kHalf, dp);
+          tmem_wait_ld();
+          const int lim = (c >= it.diag_first ? rl - (c - it.diag_first) * kChunk : kChunk) - rr.hf * kHalf;
+          p_ds_half(s, dp, pv, p.scale_log2, lse2, dd, lim, live);
           uint32_t u[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(s[h * 32 + 2 * e], s[h * 32 + 2 * e + 1]);
-          tmem_st16(cs + h * 16, u);
+          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(s[2 * e], s[2 * e + 1]);
+          tmem_st16(cs, u);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(S::kBDS + (g & 1)));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(S::kBDS + (g & 1)));
-      }
-      if (!ok) break;
-      ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBAcc + (xi & 1)), uint32_t(xi >> 1) & 1u));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t acc = lane_base + S::kColQ + uint32_t(xi & 1) * HD;
-#pragma unroll 1
-      for (int a = 0; a < HD / 32; ++a) {
-        float v[32];
-        tmem_ld32(acc + a * 32, v);
+        if (!ok) break;
+        // prefetch the next item's row values
+        if (__all_sync(0xffffffffu, ctl.wait(bar(S::kBItem + (k + 1) % kRing), uint32_t((k + 1) / kRing) & 1u))) {
+          const DqSlot nx = read_slot(ring, k + 1);
+          if (!nx.last) {
+            int nh, nt;
+            const bool nreal = tile_row<BLK>(p, QTile{nx.i, nx.h0}, rr.r, nh, nt);
+            const size_t nrow = size_t(nh) * p.n + (nreal ? nt : 0);
+            nlse2 = nreal ? p.lse[nrow] * kLog2e : 0.f;
+            ndd = nreal ? p.dsum[nrow] : 0.f;
+            have_next = true;
+          }
+        }
+        ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBAcc + (xi & 1)), uint32_t(xi >> 1) & 1u));
+        if (!ok) break;
+        tc_fence_after();
+        float v[kCols];
+        const uint32_t acc = rr.lane_base + S::kColQ + uint32_t(xi & 1) * HD + rr.hf * kCols;
+#pragma unroll
+        for (int a = 0; a < kCols / 32; ++a) tmem_ld32(acc + a * 32, v + a * 32);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(S::kBAccFree + (xi & 1)));
+        ++xi;
         if (real) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(out + a * 32 + e) =
+          for (int e = 0; e < kCols; e += 4)
+            *reinterpret_cast<float4*>(out + e) =
                 make_float4(v[e] * p.scale, v[e + 1] * p.scale, v[e + 2] * p.scale, v[e + 3] * p.scale);
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(S::kBAccFree + (xi & 1)));
-      ++xi;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(S::kBItemFree + k % kRing));
     }
   }
   tc_fence_before();
@@ -649,21 +767,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- dK, dV
-// Persistent: one CTA per SM walks work items (key/value head, query-head
-// step, 64-key chunk of a key block, column segment; longest segments first,
-// every gridDim-th).  A segment lists up to 16 query blocks whose rows keep
-// the key block (the transposed layout).  Per query tile t: S = Q K^T and
-// dP = dO V^T (M = 128 query rows) into TMEM buffer t & 1; the row threads
-// write P and dS = P (dP - D) as bf16 [query][key] tiles into shared memory;
-// then dV^T += dO^T P and dK^T += Q^T dS (M = 128 along d: A is the dO / Q
-// tile read along d, B the P / dS tile read along the keys; for d = 64 the
-// upper 64 rows of M read the neighbouring tile and are never stored) into
-// the item's accumulators (two TMEM pairs, so one item's read-out overlaps
-// the next item's products).  The sums are added into dk and dv (zeroed
-// first), as segments of one column run on several CTAs.  Tiles are
+// Persistent: one CTA per SM walks work items (key/value head, column
+// segment, query-head step, 64-key chunk of a key block; head by head,
+// longest segments first inside one, every gridDim-th).  A segment lists up to 16 query blocks whose rows keep
+// the key block (the transposed layout).  Warp 0 decodes each item into a
+// ring of shared-memory slots and loads its tiles.  Per query tile t:
+// S = Q K^T and dP = dO V^T (M = 128 query rows) into TMEM buffer t & 1; the
+// row threads write P and dS = P (dP - D) as bf16 [query][key] tiles into
+// shared memory; then dV^T += dO^T P and dK^T += Q^T dS (M = 128 along d: A
+// is the dO / Q tile read along d, B the P / dS tile read along the keys; for
+// d = 64 the upper 64 rows of M read the neighbouring tile and are never
+// stored) into the item's accumulators (two TMEM pairs, so one item's
+// read-out overlaps the next item's products).  An item that holds a whole
+// column, when each key/value head has a single head step, stores its sums;
+// otherwise they are added into dk and dv (cleared first).  Tiles are
 // numbered across the CTA's items: a tile's Q and dO sit in buffer t & 1
-// until its dV / dK products are done; an item's K and V in buffer (item & 1)
-// until its last S / dP are done.
+// until its dV / dK products are done; an item's K and V in buffer
+// (item & 1) until its last S / dP are done.
 template <int BLK, int HD>
 struct DkvShape {
   static constexpr int kQBytes = kTileM * HD * 2;
@@ -674,10 +794,12 @@ struct DkvShape {
   static constexpr int kOffKV = 4 * kQBytes;               // Q, dO of buffer b at b * 2 * kQBytes
   static constexpr int kOffP = kOffKV + 4 * kTile;         // K, V of buffer b at kOffKV + b * 2 * kTile
   static constexpr int kOffBar = kOffP + 2 * kPBytes;      // P, dS
-  // kv_full[2] kv_free[2] q_full[2] s_full[2] pds_full done[2] acc_full[2] acc_free[2] drain
   static constexpr int kBKV = 0, kBKVFree = 2, kBQ = 4, kBS = 6, kBPDS = 8, kBDone = 9, kBAcc = 11,
-                       kBAccFree = 13, kBDrain = 15, kNumBars = 16;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+                       kBAccFree = 13, kBItem = 15, kBItemFree = 15 + kRing, kBDrain = 15 + 2 * kRing,
+                       kNumBars = 16 + 2 * kRing;
+  static constexpr int kSlotBytes = 96;                    // 8 ints + 16 query blocks
+  static constexpr int kOffRing = ((kOffBar + kNumBars * 8 + 15) / 16) * 16;
+  static constexpr int kOffMisc = kOffRing + kRing * kSlotBytes;
   static constexpr int kSmem = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColAcc = 256;   // acc pair b: dV at 256 + 128 b, dK 64 further
   static constexpr uint32_t kIdescS = idesc_bf16(kTileM, kChunk, 0, 0);
@@ -685,57 +807,57 @@ struct DkvShape {
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
-struct DkvItem {
-  int kvh, h0, j, key0, e0, total;
+struct DkvSlot {
+  int kvh, h0, j, key0, total, sole, last;
 };
 
 template <int BLK>
-__device__ __forceinline__ bool dkv_item(const Params& p, int x, DkvItem& it) {
+__device__ __forceinline__ bool dkv_decode(const Params& p, int x, DkvSlot& s, int& e0) {
   constexpr int CPB = BLK / kChunk;
+  // key/value head by key/value head (the Q / dO tiles in flight stay in
+  // L2), longest segment first inside a head
   const int inner = p.n_steps * CPB;
-  const int rank = x / (p.kv_heads * inner);
-  int rem = x - rank * (p.kv_heads * inner);
-  it.kvh = rem / inner;
-  rem -= it.kvh * inner;
+  const int per_head = p.items / p.kv_heads;     // segment ranks x inner
+  s.kvh = x / per_head;
+  int rem = x - s.kvh * per_head;
+  const int rank = rem / inner;
+  rem -= rank * inner;
   const int hs = rem / CPB, hh = rem - hs * CPB;
-  it.h0 = it.kvh * p.group + hs * p.pack;
-  const int lh = it.h0 % p.L;
+  s.h0 = s.kvh * p.group + hs * p.pack;
+  const int lh = s.h0 % p.L;
   const int seg = p.seg_ptr[lh] + rank;
   if (seg >= p.seg_ptr[lh + 1]) return false;
-  it.j = p.segs[3 * seg];
-  it.e0 = p.segs[3 * seg + 1];
-  it.total = p.segs[3 * seg + 2];
-  it.key0 = it.j * BLK + hh * kChunk;
+  s.j = p.segs[3 * seg];
+  e0 = p.segs[3 * seg + 1];
+  s.total = p.segs[3 * seg + 2];
+  s.key0 = s.j * BLK + hh * kChunk;
+  const int col_len = p.col_ptr[size_t(lh) * p.nb + s.j + 1] - p.col_ptr[size_t(lh) * p.nb + s.j];
+  s.sole = (p.n_steps == 1 && col_len == s.total) ? 1 : 0;
+  s.last = 0;
   return true;
 }
 
+__device__ __forceinline__ DkvSlot read_dkv_slot(const uint8_t* ring, int k, int slot_bytes) {
+  const volatile int* v = reinterpret_cast<const volatile int*>(ring + (k % kRing) * slot_bytes);
+  DkvSlot s;
+  s.kvh = v[0];
+  s.h0 = v[1];
+  s.j = v[2];
+  s.key0 = v[3];
+  s.total = v[4];
+  s.sole = v[5];
+  s.last = v[6];
+  return s;
+}
+__device__ __forceinline__ int slot_tile(const uint8_t* ring, int k, int slot_bytes, int e) {
+  return reinterpret_cast<const volatile int*>(ring + (k % kRing) * slot_bytes)[8 + e];
+}
+
 struct DkvCursor {
-  int x, e, t, y;
-  DkvItem it;
+  int k, e, t, y;
+  DkvSlot it;
   bool valid;
 };
-
-template <int BLK>
-__device__ __forceinline__ void dkv_seek(const Params& p, DkvCursor& k) {
-  while (k.x < p.items) {
-    if (dkv_item<BLK>(p, k.x, k.it)) {
-      k.valid = true;
-      return;
-    }
-    k.x += gridDim.x;
-  }
-  k.valid = false;
-}
-
-template <int BLK>
-__device__ __forceinline__ void dkv_advance(const Params& p, DkvCursor& k) {
-  ++k.t;
-  if (++k.e < k.it.total) return;
-  k.e = 0;
-  ++k.y;
-  k.x += gridDim.x;
-  dkv_seek<BLK>(p, k);
-}
 
 template <int BLK, int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -754,14 +876,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sQ = [&](int t) { return base + uint32_t(t & 1) * 2 * S::kQBytes; };
   auto sKV = [&](int y) { return base + S::kOffKV + uint32_t(y & 1) * 2 * S::kTile; };
   const uint32_t sP = base + S::kOffP, sDS = sP + S::kPBytes;
+  uint8_t* ring = smem_raw + S::kOffRing;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem_raw + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + S::kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const Ctl ctl{abort_flag, p.status, p.timeout_ns};
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < S::kNumBars; ++b)
-      mbar_init(bar(b), (b == S::kBPDS || b == S::kBAccFree || b == S::kBAccFree + 1) ? 128u : 1u);
+    for (int b = 0; b < S::kNumBars; ++b) {
+      uint32_t count = 1;
+      if (b == S::kBPDS || b == S::kBAccFree || b == S::kBAccFree + 1) count = kRowThreads;
+      if (b >= S::kBItemFree && b < S::kBItemFree + kRing) count = kRowWarps + 1;
+      mbar_init(bar(b), count);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -775,25 +902,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
-    // ---- loads
+    // ---- item ring and loads
     if (lane == 0) {
       bool ok = true;
       int t = 0, y = 0;
-      DkvItem it;
-      for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
-        if (!dkv_item<BLK>(p, x, it)) continue;
+      int k = 0;
+      for (int x = blockIdx.x; ok; x += gridDim.x) {
+        DkvSlot it{};
+        int e0 = 0;
+        const bool end = x >= p.items;
+        if (!end && !dkv_decode<BLK>(p, x, it, e0)) continue;
+        if (k >= kRing && !(ok = ctl.wait(bar(S::kBItemFree + k % kRing), uint32_t((k - kRing) / kRing) & 1u))) break;
+        volatile int* v = reinterpret_cast<volatile int*>(ring + (k % kRing) * S::kSlotBytes);
+        v[0] = it.kvh;
+        v[1] = it.h0;
+        v[2] = it.j;
+        v[3] = it.key0;
+        v[4] = it.total;
+        v[5] = it.sole;
+        v[6] = end ? 1 : 0;
+        for (int e = 0; e < (end ? 0 : it.total); ++e) v[8 + e] = p.row_idx[e0 + e];
+        mbar_arrive(bar(S::kBItem + k % kRing));
+        if (end) break;
         if (y >= 2 && !(ok = ctl.wait(bar(S::kBKVFree + (y & 1)), uint32_t((y - 2) >> 1) & 1u))) break;
         mbar_expect_tx(bar(S::kBKV + (y & 1)), 2 * S::kTile);
         tma_load_kv<HD>(sKV(y), &tmK, bar(S::kBKV + (y & 1)), it.key0, it.kvh);
         tma_load_kv<HD>(sKV(y) + S::kTile, &tmV, bar(S::kBKV + (y & 1)), it.key0, it.kvh);
         ++y;
-        for (int e = 0; e < it.total; ++e, ++t) {
+        for (int e = 0; e < it.total; ++e) {
           if (t >= 2 && !(ok = ctl.wait(bar(S::kBDone + (t & 1)), uint32_t((t - 2) >> 1) & 1u))) break;
-          const int i = p.row_idx[it.e0 + e];
+          const int i = v[8 + e];
           mbar_expect_tx(bar(S::kBQ + (t & 1)), 2 * S::kQBytes);
           tma_load_q<BLK, HD>(sQ(t), &tmQ, bar(S::kBQ + (t & 1)), i * BLK, it.h0);
           tma_load_q<BLK, HD>(sQ(t) + S::kQBytes, &tmDO, bar(S::kBQ + (t & 1)), i * BLK, it.h0);
+          ++t;
         }
+        ++k;
       }
       if (!ok) {
         for (int e = (t > 2 ? t - 2 : 0); e < t; ++e) wait_drain(bar(S::kBQ + (e & 1)), uint32_t(e >> 1) & 1u, kDrainNs);
@@ -803,11 +947,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---- products, issued as their inputs become ready
     if (lane == 0) {
-      DkvCursor cs{int(blockIdx.x), 0, 0, 0, {}, false}, cd{int(blockIdx.x), 0, 0, 0, {}, false};
-      dkv_seek<BLK>(p, cs);
-      dkv_seek<BLK>(p, cd);
-      uint64_t idle_since = 0;
       bool ok = true;
+      auto seek = [&](DkvCursor& cu, bool release) {
+        if (!(ok = ctl.wait(bar(S::kBItem + cu.k % kRing), uint32_t(cu.k / kRing) & 1u))) {
+          cu.valid = false;
+          return;
+        }
+        cu.it = read_dkv_slot(ring, cu.k, S::kSlotBytes);
+        if (release) mbar_arrive(bar(S::kBItemFree + cu.k % kRing));
+        cu.valid = !cu.it.last;
+      };
+      auto advance = [&](DkvCursor& cu, bool release) {
+        ++cu.t;
+        if (++cu.e < cu.it.total) return;
+        cu.e = 0;
+        ++cu.y;
+        ++cu.k;
+        seek(cu, release);
+      };
+      DkvCursor cs{0, 0, 0, 0, {}, false}, cd{0, 0, 0, 0, {}, false};
+      seek(cs, false);
+      seek(cd, true);
+      Idle idle;
       while (cd.valid && ok) {
         bool progress = false;
         // S(t), dP(t): TMEM buffer t & 1 is free once tile t - 2's dV / dK are issued
@@ -825,7 +986,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(S::kBS + (cs.t & 1)));
           if (cs.e == cs.it.total - 1) tc_commit(bar(S::kBKVFree + (cs.y & 1)));
-          dkv_advance<BLK>(p, cs);
+          advance(cs, false);
           progress = true;
         }
         // dV^T += dO^T P, dK^T += Q^T dS for tile t, once its P / dS are written
@@ -846,98 +1007,103 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(bar(S::kBDone + (cd.t & 1)));
           if (cd.e == cd.it.total - 1) tc_commit(bar(S::kBAcc + (cd.y & 1)));
-          dkv_advance<BLK>(p, cd);
+          advance(cd, true);
           progress = true;
         }
-        if (progress) {
-          idle_since = 0;
-        } else {
-          const uint64_t now = globaltimer();
-          if (idle_since == 0) idle_since = now;
-          if (*abort_flag) ok = false;
-          else if (now - idle_since > p.timeout_ns) {
-            *abort_flag = 1;
-            atomicOr(p.status, kStatusTimeout);
-            ok = false;
-          }
-        }
+        ok = ok && idle.step(progress, ctl);
       }
       tc_commit(bar(S::kBDrain));
       wait_drain(bar(S::kBDrain), 0, kDrainNs);
     }
   } else {
-    // ---- rows: P and dS per tile, then each item's dK / dV read-out
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
-    const uint32_t lane_base = tmem + (uint32_t(q4 * 32) << 16);
-    const int rl = r - (r / BLK) * BLK;
+    // ---- rows: P and dS per tile (half of the keys per thread), then each
+    // item's dV (warps 2-5) or dK (warps 6-9) read-out
+    const RowRole rr = row_role(tmem);
+    const int rl = rr.r - (rr.r / BLK) * BLK;
     bool ok = true;
     int t = 0, y = 0;
-    DkvItem it;
-    for (int x = blockIdx.x; x < p.items && ok; x += gridDim.x) {
-      if (!dkv_item<BLK>(p, x, it)) continue;
+    for (int k = 0; ok; ++k) {
+      ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBItem + k % kRing), uint32_t(k / kRing) & 1u));
+      if (!ok) break;
+      const DkvSlot it = read_dkv_slot(ring, k, S::kSlotBytes);
+      if (it.last) break;
       const int hh = (it.key0 - it.j * BLK) / kChunk;
-      for (int e = 0; e < it.total; ++e, ++t) {
-        const int i = p.row_idx[it.e0 + e];
+      // the row's lse and D for tile e + 1 are fetched while tile e is computed
+      auto row_vals = [&](int e, float& lse2, float& dd, bool& live) {
         int head, tok;
-        const bool real = tile_row<BLK>(p, QTile{i, it.h0}, r, head, tok);
+        const bool real = tile_row<BLK>(p, QTile{slot_tile(ring, k, S::kSlotBytes, e), it.h0}, rr.r, head, tok);
         const size_t rowi = size_t(head) * p.n + (real ? tok : 0);
-        const float lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
-        const float dd = real ? p.dsum[rowi] : 0.f;
+        lse2 = real ? p.lse[rowi] * kLog2e : 0.f;
+        dd = real ? p.dsum[rowi] : 0.f;
+        live = real;
+      };
+      float lse2, dd;
+      bool live;
+      row_vals(0, lse2, dd, live);
+      for (int e = 0; e < it.total; ++e, ++t) {
+        float nlse2 = 0.f, ndd = 0.f;
+        bool nlive = false;
+        if (e + 1 < it.total) row_vals(e + 1, nlse2, ndd, nlive);
+        const int i = slot_tile(ring, k, S::kSlotBytes, e);
         // causal: in the diagonal block, key (chunk offset + c) > row is dropped
-        const int lim = (i == it.j) ? rl - hh * kChunk : kChunk;
+        const int lim = ((i == it.j) ? rl - hh * kChunk : kChunk) - rr.hf * kHalf;
         ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBS + (t & 1)), uint32_t(t >> 1) & 1u));
         if (!ok) break;
         tc_fence_after();
-        float s[kChunk], dp[kChunk], pv[kChunk];
-        const uint32_t cs = lane_base + S::kColS + (t & 1) * kChunk, cdp = lane_base + S::kColDP + (t & 1) * kChunk;
-        tmem_ld32(cs, s);
-        tmem_ld32(cs + 32, s + 32);
-        tmem_ld32(cdp, dp);
-        tmem_ld32(cdp + 32, dp + 32);
+        float s[kHalf], dp[kHalf], pv[kHalf];
+        tmem_ld32(rr.lane_base + S::kColS + (t & 1) * kChunk + rr.hf * kHalf, s);
+        tmem_ld32(rr.lane_base + S::kColDP + (t & 1) * kChunk + rr.hf * kHalf, dp);
         tmem_wait_ld();
-        p_ds_row(s, dp, pv, p.scale_log2, lse2, dd, lim, real && lse2 > -INFINITY);
+        p_ds_half(s, dp, pv, p.scale_log2, lse2, dd, lim, live && lse2 > -INFINITY);
         // the P / dS tiles were last read by tile t - 1's products
         if (t >= 1) {
           ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBDone + ((t - 1) & 1)), uint32_t((t - 1) >> 1) & 1u));
           if (!ok) break;
         }
+        // row r, keys 32 hf .. 32 hf + 31 of the [query][key] tiles, 128-byte swizzled
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t off = uint32_t(r) * 128 + ((ch ^ (r & 7)) << 4);
-          st_shared_v4(sP + off, pack_bf16(pv[8 * ch], pv[8 * ch + 1]), pack_bf16(pv[8 * ch + 2], pv[8 * ch + 3]),
-                       pack_bf16(pv[8 * ch + 4], pv[8 * ch + 5]), pack_bf16(pv[8 * ch + 6], pv[8 * ch + 7]));
-          st_shared_v4(sDS + off, pack_bf16(s[8 * ch], s[8 * ch + 1]), pack_bf16(s[8 * ch + 2], s[8 * ch + 3]),
-                       pack_bf16(s[8 * ch + 4], s[8 * ch + 5]), pack_bf16(s[8 * ch + 6], s[8 * ch + 7]));
+        for (int q = 0; q < 4; ++q) {
+          const int ch = rr.hf * 4 + q;
+          const uint32_t off = uint32_t(rr.r) * 128 + ((ch ^ (rr.r & 7)) << 4);
+          st_shared_v4(sP + off, pack_bf16(pv[8 * q], pv[8 * q + 1]), pack_bf16(pv[8 * q + 2], pv[8 * q + 3]),
+                       pack_bf16(pv[8 * q + 4], pv[8 * q + 5]), pack_bf16(pv[8 * q + 6], pv[8 * q + 7]));
+          st_shared_v4(sDS + off, pack_bf16(s[8 * q], s[8 * q + 1]), pack_bf16(s[8 * q + 2], s[8 * q + 3]),
+                       pack_bf16(s[8 * q + 4], s[8 * q + 5]), pack_bf16(s[8 * q + 6], s[8 * q + 7]));
         }
         fence_proxy_async();
         tc_fence_before();
         mbar_arrive(bar(S::kBPDS));
+        lse2 = nlse2;
+        dd = ndd;
+        live = nlive;
       }
       if (!ok) break;
       // TMEM lane r holds element d = r of the chunk's 64 key rows
       ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBAcc + (y & 1)), uint32_t(y >> 1) & 1u));
       if (!ok) break;
       tc_fence_after();
-      float vk[kChunk], vv[kChunk];
-      const uint32_t accv = lane_base + S::kColAcc + uint32_t(y & 1) * 128;
-      tmem_ld32(accv + 64, vk);
-      tmem_ld32(accv + 96, vk + 32);
-      tmem_ld32(accv, vv);
-      tmem_ld32(accv + 32, vv + 32);
+      float vals[kChunk];
+      const uint32_t acc = rr.lane_base + S::kColAcc + uint32_t(y & 1) * 128 + rr.hf * 64;
+      tmem_ld32(acc, vals);
+      tmem_ld32(acc + 32, vals + 32);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(S::kBAccFree + (y & 1)));
       ++y;
-      if (r < HD) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(S::kBItemFree + k % kRing));
+      if (rr.r < HD) {
+        float* dst = rr.hf ? p.dk : p.dv;
+        const float mul = rr.hf ? p.scale : 1.f;
+        const size_t row0 = size_t(it.kvh) * p.n;
+        if (it.sole) {
 #pragma unroll
-        for (int c = 0; c < kChunk; ++c) {
-          const int key = it.key0 + c;
-          if (key < p.n) {
-            const size_t at = (size_t(it.kvh) * p.n + key) * HD + r;
-            atomicAdd(p.dk + at, vk[c] * p.scale);
-            atomicAdd(p.dv + at, vv[c]);
-          }
+          for (int c = 0; c < kChunk; ++c)
+            if (it.key0 + c < p.n) dst[(row0 + it.key0 + c) * HD + rr.r] = vals[c] * mul;
+        } else {
+#pragma unroll
+          for (int c = 0; c < kChunk; ++c)
+            if (it.key0 + c < p.n) atomicAdd(dst + (row0 + it.key0 + c) * HD + rr.r, vals[c] * mul);
         }
       }
     }
@@ -1077,10 +1243,16 @@ int launch_instance(const Launch& a, const bwd::Params& p) {
   if (st == BSA_OK) st = encode_kv(&mk, a.k, a.kv_heads, a.n, HD);
   if (st == BSA_OK) st = encode_kv(&mv, a.v, a.kv_heads, a.n, HD);
   if (st != BSA_OK) return st;
-  const size_t grad_kv = size_t(a.kv_heads) * a.n * HD * sizeof(float);
-  cudaError_t e = cudaMemsetAsync(p.dk, 0, grad_kv, a.stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(p.dv, 0, grad_kv, a.stream);
-  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing dk, dv: ") + cudaGetErrorString(e));
+  cudaError_t e = cudaSuccess;
+  if (p.n_steps == 1) {
+    // only rows that several CTAs add into, or that nothing writes, are cleared
+    bwd::bsa_bwd_clear_kernel<HD><<<a.kv_heads * p.nb, 256, 0, a.stream>>>(p, BLK);
+  } else {
+    const size_t grad_kv = size_t(a.kv_heads) * a.n * HD * sizeof(float);
+    e = cudaMemsetAsync(p.dk, 0, grad_kv, a.stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p.dv, 0, grad_kv, a.stream);
+    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing dk, dv: ") + cudaGetErrorString(e));
+  }
   const unsigned rows_grid = unsigned((a.dq_rows + 7) / 8);
   bwd::bsa_bwd_rowdot_kernel<HD><<<rows_grid, 256, 0, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.dsum, a.dq_rows);
@@ -1137,6 +1309,7 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   p.row_ptr = layout->d_row_ptr;
   p.col_idx = layout->d_col_idx;
   p.order = layout->d_order;
+  p.col_ptr = layout->d_col_ptr;
   p.row_idx = layout->d_row_idx;
   p.seg_ptr = layout->d_seg_ptr;
   p.segs = layout->d_segs;
