@@ -630,7 +630,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       Idle idle;
       while (cd.valid && ok) {
         bool progress = false;
-        if (cs.valid && cs.g < cd.g + 2 && mbar_test(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u) &&
+        if (cs.valid && cs.g < cd.g + 2 &&
+            (cs.c > 0 || mbar_test(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u)) &&
             mbar_test(bar(S::kBK + cs.g % S::kRingK), uint32_t(cs.g / S::kRingK) & 1u) &&
             mbar_test(bar(S::kBV + cs.g % S::kRingV), uint32_t(cs.g / S::kRingV) & 1u)) {
           tc_fence_after();
@@ -972,7 +973,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (cd.valid && ok) {
         bool progress = false;
         // S(t), dP(t): TMEM buffer t & 1 is free once tile t - 2's dV / dK are issued
-        if (cs.valid && cs.t < cd.t + 2 && mbar_test(bar(S::kBKV + (cs.y & 1)), uint32_t(cs.y >> 1) & 1u) &&
+        if (cs.valid && cs.t < cd.t + 2 &&
+            (cs.e > 0 || mbar_test(bar(S::kBKV + (cs.y & 1)), uint32_t(cs.y >> 1) & 1u)) &&
             mbar_test(bar(S::kBQ + (cs.t & 1)), uint32_t(cs.t >> 1) & 1u)) {
           tc_fence_after();
           const uint32_t qb = sQ(cs.t), kb = sKV(cs.y), vb = kb + S::kTile;
