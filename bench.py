@@ -315,11 +315,19 @@ def main():
     ap.add_argument("--only-device", action="store_true",
                     help="device-timed leg only (no e2e, CPU baseline or other workloads); "
                          "the form used for profiler captures")
+    ap.add_argument("--leg", default=None, choices=["backward", "bsbr"],
+                    help="time one secondary leg alone on --workload (backward) or the BSBR "
+                         "workload (bsbr) and print its JSON; the form used for profiler captures")
+    ap.add_argument("--n", type=int, default=None,
+                    help="with --leg backward: the workload's geometry at this sequence length "
+                         "(a smaller case for full profiler captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.leg is not None:
+        return run_leg(args, w)
 
     import torch
     import torch.distributed as dist
@@ -521,6 +529,28 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+    return 0
+
+
+def run_leg(args, w):
+    """One secondary leg alone (no headline, e2e or CPU legs), one JSON line."""
+    import dataclasses
+    import torch
+    import block_sparse_long_bsa_b200 as bsa
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    bsa.load_library()
+    dev = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    if args.leg == "backward":
+        if args.n is not None:
+            w = dataclasses.replace(w, n=args.n)
+        res = bench_backward(w, dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup)
+    else:
+        res = bench_bsbr(WORKLOADS["bsbr_block_diagonal"], dev, stream, flush, bsa, torch, steps=args.steps,
+                         warmup=args.warmup)
+    print(json.dumps({"leg": args.leg, "workload": w.name, "n": w.n, "result": res}), flush=True)
     return 0
 
 
