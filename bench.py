@@ -548,8 +548,8 @@ def run_leg(args, w):
             w = dataclasses.replace(w, n=args.n)
         res = bench_backward(w, dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup)
     else:
-        res = bench_bsbr(WORKLOADS["bsbr_block_diagonal"], dev, stream, flush, bsa, torch, steps=args.steps,
-                         warmup=args.warmup)
+        w = WORKLOADS["bsbr_block_diagonal"]
+        res = bench_bsbr(w, dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup)
     print(json.dumps({"leg": args.leg, "workload": w.name, "n": w.n, "result": res}), flush=True)
     return 0
 
