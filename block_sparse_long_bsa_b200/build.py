@@ -22,8 +22,9 @@ NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 CU_SOURCES = ["bsa_fwd_sm100a.cu", "bsa_noalloc.cu", "bsa_decode.cu", "bsa_bwd_sm100a.cu", "bsa_bsbr_sm100a.cu"]
-CPP_SOURCES = ["bsa_api.cpp", "bsa_layout.cpp"]
-HEADERS = [os.path.join(INCLUDE, "bsa.h"), os.path.join(CSRC, "bsa_internal.h")]
+CPP_SOURCES = ["bsa_api.cpp", "bsa_layout.cpp", "bsa_tmap.cpp"]
+HEADERS = [os.path.join(INCLUDE, "bsa.h"), os.path.join(CSRC, "bsa_internal.h"), os.path.join(CSRC, "bsa_device.cuh"),
+           os.path.join(CSRC, "bsa_tmap.h")]
 
 
 def _newer(target: str, deps) -> bool:
