@@ -193,35 +193,40 @@ __global__ void __launch_bounds__(256) bsa_bwd_clear_kernel(const Params p, int 
 
 // ---------------------------------------------------------------- dQ
 // Persistent: one CTA per SM walks query tiles (head group by head group,
-// longest row first inside one, every gridDim-th).  Warp 0 decodes each tile into a ring of shared-memory slots
-// (read by the other warps) and loads its Q, dO, K and V tiles.  Per 64-key
-// chunk c of a tile's kept blocks: S = Q K_c^T and dP = dO V_c^T into TMEM
-// buffer c & 1; the row threads turn them into dS = P (dP - D), rounded to
-// bf16 and packed over their own S columns; then dQ += dS K_c (A = dS read
-// from TMEM, B = K_c read along d) into the tile's accumulator (two TMEM
+// longest row first inside one, every gridDim-th).  Warp 0 decodes each tile
+// into a ring of shared-memory slots (read by the other warps) and loads its
+// Q, dO, K and V tiles.  A tile's kept blocks are taken 128 keys at a time
+// (two 64-key chunks: two blocks for B = 64, one for B = 128; a lone last
+// chunk is paired with zero rows): S = Q K^T and dP = dO V^T as N = 128
+// products into single TMEM buffers; the row threads (two per row, 64 keys
+// each) read both, release S, turn them into dS = P (dP - D), rounded to bf16
+// and packed over the dP columns they read; then dQ += dS K (A = dS read from
+// TMEM, B = K read along d) into the tile's accumulator (two TMEM
 // accumulators, so one tile's read-out overlaps the next tile's products).
-// Chunks are numbered across the CTA's tiles: K_c sits in slot c % 4 until
-// dQ_c is done, V_c in slot c % 2 until S_c / dP_c are done, and a tile's Q
-// and dO in buffer (tile & 1) until its last S / dP are done.
+// The products go S(s + 1), dQ(s), dP(s + 1): the next scores are formed while
+// the row threads work on the current ones.  Steps are numbered across the
+// CTA's tiles: K of step s sits in slot s % 2 until dQ(s) is done, V in the
+// single V slot until dP(s) is done, a tile's Q and dO in buffer (tile & 1)
+// until its last dP is done.
 template <int BLK, int HD>
 struct DqShape {
   static constexpr int kCPB = BLK / kChunk;
+  static constexpr int kStep = 2 * kChunk;                 // keys per step
   static constexpr int kQBytes = kTileM * HD * 2;
-  static constexpr int kTile = kChunk * HD * 2;
+  static constexpr int kKV = kStep * HD * 2;               // one step's K (or V): [atom][128 rows][64 columns]
   static constexpr int kAtomQ = kTileM * 128;
-  static constexpr int kAtomKV = kChunk * 128;
-  static constexpr int kRingK = 4, kRingV = 2;
+  static constexpr int kAtomKV = kStep * 128;
   static constexpr int kOffK = 4 * kQBytes;                // Q, dO of buffer b at b * 2 * kQBytes
-  static constexpr int kOffV = kOffK + kRingK * kTile;
-  static constexpr int kOffBar = kOffV + kRingV * kTile;
-  static constexpr int kBQ = 0, kBQFree = 2, kBK = 4, kBKFree = 8, kBV = 12, kBS = 14, kBDS = 16, kBAcc = 18,
-                       kBAccFree = 20, kBItem = 22, kBItemFree = 22 + kRing, kBDrain = 22 + 2 * kRing,
-                       kNumBars = 23 + 2 * kRing;
+  static constexpr int kOffV = kOffK + 2 * kKV;
+  static constexpr int kOffBar = kOffV + kKV;
+  static constexpr int kBQ = 0, kBQFree = 2, kBK = 4, kBKFree = 6, kBV = 8, kBS = 9, kBDP = 10, kBRead = 11,
+                       kBDS = 12, kBAcc = 13, kBAccFree = 15, kBItem = 17, kBItemFree = 17 + kRing,
+                       kBDrain = 17 + 2 * kRing, kNumBars = 18 + 2 * kRing;
   static constexpr int kOffRing = ((kOffBar + kNumBars * 8 + 15) / 16) * 16;
   static constexpr int kOffMisc = kOffRing + kRing * 32;
   static constexpr int kSmem = kOffMisc + 16;
   static constexpr int kColS = 0, kColDP = 128, kColQ = 256;
-  static constexpr uint32_t kIdescS = idesc_bf16(kTileM, kChunk, 0, 0);
+  static constexpr uint32_t kIdescS = idesc_bf16(kTileM, kStep, 0, 0);
   static constexpr uint32_t kIdescDQ = idesc_bf16(kTileM, HD, 0, 1);
   static_assert(kSmem <= 227 * 1024, "shared memory");
   static_assert(kColQ + 2 * HD <= 512, "TMEM columns");
@@ -273,13 +278,15 @@ __device__ __forceinline__ DqSlot read_slot(const uint8_t* ring, int k) {
   return s;
 }
 
-// A position in a CTA's stream of chunks: ring item k, chunk c of it, global
-// chunk number g, and the count of non-empty items before it.
+// A position in a CTA's stream of steps: ring item k, step c of it, global
+// step number g, and the count of non-empty items before it.
 struct DqCursor {
   int k, c, g, xi;
   DqSlot it;
   bool valid;
 };
+
+__device__ __forceinline__ int dq_steps(const DqSlot& it) { return (it.nch + 1) >> 1; }
 
 template <int BLK, int HD>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -297,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar0 = base + S::kOffBar;
   auto bar = [&](int idx) { return bar0 + 8u * uint32_t(idx); };
   auto sQ = [&](int b) { return base + uint32_t(b) * 2 * S::kQBytes; };
-  auto sK = [&](int g) { return base + S::kOffK + uint32_t(g % S::kRingK) * S::kTile; };
-  auto sV = [&](int g) { return base + S::kOffV + uint32_t(g % S::kRingV) * S::kTile; };
+  auto sK = [&](int g) { return base + S::kOffK + uint32_t(g & 1) * S::kKV; };
+  const uint32_t sV = base + S::kOffV;
   uint8_t* ring = smem_raw + S::kOffRing;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(smem_raw + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem_raw + S::kOffMisc + 4);
@@ -308,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int b = 0; b < S::kNumBars; ++b) {
       uint32_t count = 1;
-      if (b == S::kBDS || b == S::kBDS + 1 || b == S::kBAccFree || b == S::kBAccFree + 1) count = kRowThreads;
+      if (b == S::kBRead || b == S::kBDS || b == S::kBAccFree || b == S::kBAccFree + 1) count = kRowThreads;
       if (b >= S::kBItemFree && b < S::kBItemFree + kRing) count = kRowWarps + 1;
       mbar_init(bar(b), count);
     }
@@ -328,7 +335,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- item ring and loads
     if (lane == 0) {
       bool ok = true;
-      int nk = 0, nv = 0, xi = 0;   // K, V and Q / dO loads issued (chunk g's K is load g)
+      int nk = 0, nv = 0, xi = 0;   // K, V and Q / dO loads issued (step g's K is load g)
+      // one step's K or V: for each 64-key half and 64-column atom, one box
+      // landing at [atom][half * 64 + row][64 columns]; a half past the
+      // tile's chunks reads rows at n (zero-filled)
+      auto load_step = [&](uint32_t dst, const CUtensorMap* m, uint32_t b, const DqSlot& it, int step) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int c = 2 * step + h;
+          const int key0 = c < it.nch ? p.col_idx[it.start + c / CPB] * BLK + (c % CPB) * kChunk : p.n;
+#pragma unroll
+          for (int a = 0; a < HD / 64; ++a)
+            tma_load_3d(dst + a * S::kAtomKV + h * kChunk * 128, m, b, a * 64, key0, it.kvh);
+        }
+      };
       for (int k = 0, x = blockIdx.x; ok; ++k, x += gridDim.x) {
         if (k >= kRing && !(ok = ctl.wait(bar(S::kBItemFree + k % kRing), uint32_t((k - kRing) / kRing) & 1u))) break;
         const DqSlot it = dq_decode<BLK>(p, x);
@@ -349,34 +369,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_q<BLK, HD>(sQ(b), &tmQ, bar(S::kBQ + b), it.i * BLK, it.h0);
         tma_load_q<BLK, HD>(sQ(b) + S::kQBytes, &tmDO, bar(S::kBQ + b), it.i * BLK, it.h0);
         ++xi;
-        for (int c = 0; c < it.nch; ++c) {
+        for (int st = 0; st < dq_steps(it); ++st) {
           const int g = nk;
-          const int key0 = p.col_idx[it.start + c / CPB] * BLK + (c % CPB) * kChunk;
-          // K slot g % 4 held chunk g - 4 until its dQ product; V slot g % 2
-          // held chunk g - 2 until its S / dP products
-          if (g >= S::kRingK &&
-              !(ok = ctl.wait(bar(S::kBKFree + g % S::kRingK), uint32_t((g - S::kRingK) / S::kRingK) & 1u)))
-            break;
-          mbar_expect_tx(bar(S::kBK + g % S::kRingK), S::kTile);
-          tma_load_kv<HD>(sK(g), &tmK, bar(S::kBK + g % S::kRingK), key0, it.kvh);
+          // K slot g % 2 held step g - 2 until its dQ product; the V slot held
+          // step g - 1 until its dP product
+          if (g >= 2 && !(ok = ctl.wait(bar(S::kBKFree + (g & 1)), uint32_t((g - 2) >> 1) & 1u))) break;
+          mbar_expect_tx(bar(S::kBK + (g & 1)), S::kKV);
+          load_step(sK(g), &tmK, bar(S::kBK + (g & 1)), it, st);
           ++nk;
-          if (g >= S::kRingV && !(ok = ctl.wait(bar(S::kBS + (g & 1)), uint32_t((g - S::kRingV) >> 1) & 1u))) break;
-          mbar_expect_tx(bar(S::kBV + g % S::kRingV), S::kTile);
-          tma_load_kv<HD>(sV(g), &tmV, bar(S::kBV + g % S::kRingV), key0, it.kvh);
+          if (g >= 1 && !(ok = ctl.wait(bar(S::kBDP), uint32_t(g - 1) & 1u))) break;
+          mbar_expect_tx(bar(S::kBV), S::kKV);
+          load_step(sV, &tmV, bar(S::kBV), it, st);
           ++nv;
         }
       }
       if (!ok) {
         // let the copies in flight land before the CTA exits
-        for (int e = (nk > S::kRingK ? nk - S::kRingK : 0); e < nk; ++e)
-          wait_drain(bar(S::kBK + e % S::kRingK), uint32_t(e / S::kRingK) & 1u, kDrainNs);
-        for (int e = (nv > S::kRingV ? nv - S::kRingV : 0); e < nv; ++e)
-          wait_drain(bar(S::kBV + e % S::kRingV), uint32_t(e / S::kRingV) & 1u, kDrainNs);
+        for (int e = (nk > 2 ? nk - 2 : 0); e < nk; ++e) wait_drain(bar(S::kBK + (e & 1)), uint32_t(e >> 1) & 1u, kDrainNs);
+        if (nv > 0) wait_drain(bar(S::kBV), uint32_t(nv - 1) & 1u, kDrainNs);
         for (int e = (xi > 2 ? xi - 2 : 0); e < xi; ++e) wait_drain(bar(S::kBQ + (e & 1)), uint32_t(e >> 1) & 1u, kDrainNs);
       }
     }
   } else if (warp == 1) {
-    // ---- products, issued as their inputs become ready
+    // ---- products
     if (lane == 0) {
       bool ok = true;
       // cursor load: the next non-empty item from ring item k on; the dQ
@@ -400,60 +415,87 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto advance = [&](DqCursor& cu, bool release) {
         ++cu.g;
-        if (++cu.c < cu.it.nch) return;
+        if (++cu.c < dq_steps(cu.it)) return;
         cu.c = 0;
         ++cu.xi;
         ++cu.k;
         seek(cu, release);
       };
-      DqCursor cs{0, 0, 0, 0, {}, false}, cd{0, 0, 0, 0, {}, false};
-      seek(cs, false);
+      // S of step s (cursor cs) into the S buffer, once its K (and, for a
+      // tile's first step, Q) have landed
+      auto issue_s = [&](const DqCursor& cs) -> bool {
+        if ((cs.c == 0 && !ctl.wait(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u)) ||
+            !ctl.wait(bar(S::kBK + (cs.g & 1)), uint32_t(cs.g >> 1) & 1u))
+          return false;
+        tc_fence_after();
+        const uint32_t qb = sQ(cs.xi & 1), kb = sK(cs.g);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
+          mma_ss(tmem + S::kColS, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
+        }
+        tc_commit(bar(S::kBS));
+        return true;
+      };
+      // dP of step s into the dP buffer, once its V has landed
+      auto issue_dp = [&](const DqCursor& cs) -> bool {
+        if (!ctl.wait(bar(S::kBV), uint32_t(cs.g) & 1u)) return false;
+        tc_fence_after();
+        const uint32_t qb = sQ(cs.xi & 1) + S::kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
+          mma_ss(tmem + S::kColDP, sw128_desc(qb + ao, 16, 1024), sw128_desc(sV + bo, 16, 1024), S::kIdescS, kk > 0);
+        }
+        tc_commit(bar(S::kBDP));
+        if (cs.c == dq_steps(cs.it) - 1) tc_commit(bar(S::kBQFree + (cs.xi & 1)));   // last reader of Q, dO
+        return true;
+      };
+      DqCursor cd{0, 0, 0, 0, {}, false};
       seek(cd, true);
-      Idle idle;
-      while (cd.valid && ok) {
-        bool progress = false;
-        if (cs.valid && cs.g < cd.g + 2 &&
-            (cs.c > 0 || mbar_test(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u)) &&
-            mbar_test(bar(S::kBK + cs.g % S::kRingK), uint32_t(cs.g / S::kRingK) & 1u) &&
-            mbar_test(bar(S::kBV + cs.g % S::kRingV), uint32_t(cs.g / S::kRingV) & 1u)) {
-          tc_fence_after();
-          const uint32_t qb = sQ(cs.xi & 1), kb = sK(cs.g), vb = sV(cs.g);
-          const uint32_t ds = tmem + S::kColS + (cs.g & 1) * kChunk, ddp = tmem + S::kColDP + (cs.g & 1) * kChunk;
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
-            mma_ss(ds, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
-            mma_ss(ddp, sw128_desc(qb + S::kQBytes + ao, 16, 1024), sw128_desc(vb + bo, 16, 1024), S::kIdescS,
-                   kk > 0);
+      if (cd.valid) ok = issue_s(cd) && issue_dp(cd);
+      while (ok && cd.valid) {
+        DqCursor nx = cd;                      // the next step (same item or the next one)
+        {
+          ++nx.g;
+          if (++nx.c >= dq_steps(nx.it)) {
+            nx.c = 0;
+            ++nx.xi;
+            ++nx.k;
+            seek(nx, false);
           }
-          tc_commit(bar(S::kBS + (cs.g & 1)));
-          if (cs.c == cs.it.nch - 1) tc_commit(bar(S::kBQFree + (cs.xi & 1)));
-          advance(cs, false);
-          progress = true;
         }
-        if ((cd.g < cs.g || !cs.valid) && mbar_test(bar(S::kBDS + (cd.g & 1)), uint32_t(cd.g >> 1) & 1u) &&
-            (cd.c > 0 || cd.xi < 2 ||
-             mbar_test(bar(S::kBAccFree + (cd.xi & 1)), uint32_t((cd.xi - 2) >> 1) & 1u))) {
-          tc_fence_after();
-          // dS of keys 0-31 is packed at columns 0-15 of the S buffer, keys 32-63 at 32-47
-          const uint32_t pa = tmem + S::kColS + (cd.g & 1) * kChunk, kb = sK(cd.g);
+        // the row threads have read S(s) and dP(s): S(s + 1) may overwrite S
+        if (!(ok = ctl.wait(bar(S::kBRead), uint32_t(cd.g) & 1u))) break;
+        if (nx.valid && !(ok = issue_s(nx))) break;
+        // dQ(s) once dS(s) is in TMEM (and, for a tile's first step, its
+        // accumulator has been read out for the tile two before)
+        if (!(ok = ctl.wait(bar(S::kBDS), uint32_t(cd.g) & 1u))) break;
+        if (cd.c == 0 && cd.xi >= 2 &&
+            !(ok = ctl.wait(bar(S::kBAccFree + (cd.xi & 1)), uint32_t((cd.xi - 2) >> 1) & 1u)))
+          break;
+        tc_fence_after();
+        {
+          const uint32_t kb = sK(cd.g);
           const uint32_t acc = tmem + S::kColQ + uint32_t(cd.xi & 1) * HD;
+          // dS of keys 64 h + 16 j (j < 4) is packed at dP columns 64 h + 8 j
 #pragma unroll
-          for (int kk = 0; kk < kChunk / 16; ++kk)
-            mma_ts(acc, pa + (kk >> 1) * 32 + (kk & 1) * 8, sw128_desc(kb + kk * 16 * 128, S::kAtomKV, 1024),
-                   S::kIdescDQ, (cd.c > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar(S::kBKFree + cd.g % S::kRingK));
-          if (cd.c == cd.it.nch - 1) tc_commit(bar(S::kBAcc + (cd.xi & 1)));
-          advance(cd, true);
-          progress = true;
+          for (int kk = 0; kk < S::kStep / 16; ++kk)
+            mma_ts(acc, tmem + S::kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
+                   sw128_desc(kb + kk * 16 * 128, S::kAtomKV, 1024), S::kIdescDQ, (cd.c > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar(S::kBKFree + (cd.g & 1)));
+          if (cd.c == dq_steps(cd.it) - 1) tc_commit(bar(S::kBAcc + (cd.xi & 1)));
         }
-        ok = ok && idle.step(progress, ctl);
+        // dP(s + 1) overwrites the dP buffer after dQ(s) has read it (same queue)
+        if (nx.valid && !(ok = issue_dp(nx))) break;
+        advance(cd, true);
       }
       tc_commit(bar(S::kBDrain));
       wait_drain(bar(S::kBDrain), 0, kDrainNs);
     }
   } else {
-    // ---- rows: dS, then each tile's dQ read-out (half of the columns per thread)
+    // ---- rows: dS, then each tile's dQ read-out (half of the keys and of the
+    // dQ columns per thread)
     const RowRole rr = row_role(tmem);
     const int rl = rr.r - (rr.r / BLK) * BLK;
     constexpr int kCols = HD / 2;
@@ -487,24 +529,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         const bool live = real && lse2 > -INFINITY;
-        for (int c = 0; c < it.nch; ++c, ++g) {
-          ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBS + (g & 1)), uint32_t(g >> 1) & 1u));
+        const int steps = dq_steps(it);
+        for (int st = 0; st < steps; ++st, ++g) {
+          ok = __all_sync(0xffffffffu, ctl.wait(bar(S::kBS), uint32_t(g) & 1u) && ctl.wait(bar(S::kBDP), uint32_t(g) & 1u));
           if (!ok) break;
           tc_fence_after();
-          float s[kHalf], dp[kHalf], pv[kHalf];
-          const uint32_t cs = rr.lane_base + S::kColS + (g & 1) * kChunk + rr.hf * kHalf;
+          float s[kChunk], dp[kChunk];
+          const uint32_t cs = rr.lane_base + S::kColS + rr.hf * kChunk;
+          const uint32_t cdp = rr.lane_base + S::kColDP + rr.hf * kChunk;
           tmem_ld32(cs, s);
-          tmem_ld32(rr.lane_base + S::kColDP + (g & 1) * kChunk + rr.hf * kHalf, dp);
+          tmem_ld32(cs + 32, s + 32);
+          tmem_ld32(cdp, dp);
+          tmem_ld32(cdp + 32, dp + 32);
           tmem_wait_ld();
-          const int lim = (c >= it.diag_first ? rl - (c - it.diag_first) * kChunk : kChunk) - rr.hf * kHalf;
-          p_ds_half(s, dp, pv, p.scale_log2, lse2, dd, lim, live);
-          uint32_t u[16];
+          tc_fence_before();
+          mbar_arrive(bar(S::kBRead));
+          // keys of chunk c = 2 st + hf: none past the tile's chunks; in the
+          // diagonal block, key (chunk offset + j) > row is dropped
+          const int c = 2 * st + rr.hf;
+          const int lim = c >= it.nch ? -1 : (c >= it.diag_first ? rl - (c - it.diag_first) * kChunk : kChunk);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) u[e] = pack_bf16(s[2 * e], s[2 * e + 1]);
-          tmem_st16(cs, u);
+          for (int j = 0; j < kChunk; ++j) {
+            const bool keep = live && j <= lim;
+            const float pr = keep ? ex2(fmaf(s[j], p.scale_log2, -lse2)) : 0.f;
+            s[j] = pr * (dp[j] - dd);
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t u[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) u[e] = pack_bf16(s[h * 32 + 2 * e], s[h * 32 + 2 * e + 1]);
+            tmem_st16(cdp + h * 16, u);
+          }
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(bar(S::kBDS + (g & 1)));
+          mbar_arrive(bar(S::kBDS));
         }
         if (!ok) break;
         // prefetch the next item's row values
@@ -953,10 +1012,15 @@ int launch_instance(const Launch& a, const bwd::Params& p) {
   std::memset(&mdo, 0, sizeof(mdo));
   std::memset(&mk, 0, sizeof(mk));
   std::memset(&mv, 0, sizeof(mv));
+  CUtensorMap mk2, mv2;   // the dq kernel's K and V: 64-row x 64-column boxes, one per atom
+  std::memset(&mk2, 0, sizeof(mk2));
+  std::memset(&mv2, 0, sizeof(mv2));
   st = encode_q(&mq, a.q, a.heads, a.n, HD, BLK);
   if (st == BSA_OK) st = encode_q(&mdo, a.dout, a.heads, a.n, HD, BLK);
   if (st == BSA_OK) st = encode_kv(&mk, a.k, a.kv_heads, a.n, HD);
   if (st == BSA_OK) st = encode_kv(&mv, a.v, a.kv_heads, a.n, HD);
+  if (st == BSA_OK) st = encode_atoms(&mk2, a.k, a.kv_heads, a.n, HD, 64);
+  if (st == BSA_OK) st = encode_atoms(&mv2, a.v, a.kv_heads, a.n, HD, 64);
   if (st != BSA_OK) return st;
   cudaError_t e = cudaSuccess;
   if (p.n_steps == 1) {
@@ -974,7 +1038,7 @@ int launch_instance(const Launch& a, const bwd::Params& p) {
   bwd::Params pq = p, pk = p;
   pq.items = a.items_dq;
   pk.items = a.items_dkv;
-  if (a.items_dq > 0) kq<<<a.items_dq < a.sms ? a.items_dq : a.sms, bwd::kThreads, smem_q, a.stream>>>(mq, mdo, mk, mv, pq);
+  if (a.items_dq > 0) kq<<<a.items_dq < a.sms ? a.items_dq : a.sms, bwd::kThreads, smem_q, a.stream>>>(mq, mdo, mk2, mv2, pq);
   if (a.items_dkv > 0)
     kkv<<<a.items_dkv < a.sms ? a.items_dkv : a.sms, bwd::kThreads, smem_kv, a.stream>>>(mq, mdo, mk, mv, pk);
   e = cudaGetLastError();

@@ -75,6 +75,13 @@ int encode_q(CUtensorMap* m, const void* ptr, int heads, int n, int d, int blk) 
   return encode_tiled(m, ptr, 3, dims, str, box);
 }
 
+int encode_atoms(CUtensorMap* m, const void* ptr, int slices, int n, int d, int rows) {
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(slices)};
+  const cuuint64_t str[2] = {cuuint64_t(d) * 2, cuuint64_t(n) * cuuint64_t(d) * 2};
+  const cuuint32_t box[3] = {64, cuuint32_t(rows), 1};
+  return encode_tiled(m, ptr, 3, dims, str, box);
+}
+
 int encode_o(CUtensorMap* m, const void* ptr, int heads, int n, int d) {
   const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(heads)};
   const cuuint64_t str[2] = {cuuint64_t(d) * 2, cuuint64_t(n) * cuuint64_t(d) * 2};

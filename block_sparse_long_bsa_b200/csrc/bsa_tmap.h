@@ -27,6 +27,11 @@ inline int encode_kv(CUtensorMap* m, const void* ptr, int slices, int n, int d) 
 // dimension inside the atom dimension), landing as [atom][128 rows][64 columns].
 int encode_q(CUtensorMap* m, const void* ptr, int heads, int n, int d, int blk);
 
+// [slices][n][d] bf16 in boxes of `rows` rows x 64 columns of one slice (the
+// column coordinate picks the 64-column atom), so several boxes can be
+// placed as [atom][rows of several blocks][64 columns].
+int encode_atoms(CUtensorMap* m, const void* ptr, int slices, int n, int d, int rows);
+
 // o [heads][n][d] for stores: one warp's 32 rows x 64 columns per box.
 int encode_o(CUtensorMap* m, const void* ptr, int heads, int n, int d);
 
