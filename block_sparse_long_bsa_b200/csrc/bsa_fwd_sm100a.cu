@@ -400,14 +400,15 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         };
         auto issue_pv = [&](int q) -> bool {
           const int c = c0 + q;
-          if (!ctl.wait(bPFull(c), parS(c))) return false;
-          tc_fence_after();
+          // V and the O hand-over first: they are normally ready long before
+          // the softmax hands over P, so their barrier tests do not sit
+          // between P and the products
+          if (!ctl.wait(bVFull(c), parV(c))) return false;
           if (q == 0 && k > 0) {
             // the previous item's epilogue has read O out of TMEM
             if (!ctl.wait(bOFree, (k - 1) & 1)) return false;
-            tc_fence_after();
           }
-          if (!ctl.wait(bVFull(c), parV(c))) return false;
+          if (!ctl.wait(bPFull(c), parS(c))) return false;
           tc_fence_after();
           const uint32_t pa = tmem + S::kColS + (c & 1) * kChunk;
           const uint32_t vb = sV + (c % kVSlots) * S::kTileBytes;
