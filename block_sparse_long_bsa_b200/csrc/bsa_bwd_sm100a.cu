@@ -421,12 +421,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++cu.k;
         seek(cu, release);
       };
-      // S of step s (cursor cs) into the S buffer, once its K (and, for a
-      // tile's first step, Q) have landed
-      auto issue_s = [&](const DqCursor& cs) -> bool {
-        if ((cs.c == 0 && !ctl.wait(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u)) ||
-            !ctl.wait(bar(S::kBK + (cs.g & 1)), uint32_t(cs.g >> 1) & 1u))
-          return false;
+      // Every wait for a load (or an accumulator hand-back) is taken before
+      // the wait for the row threads that precedes the product, so no
+      // barrier test sits between the row threads' hand-over and the
+      // product (the tensor core's instruction queue is short).
+      auto loads_s = [&](const DqCursor& cs) -> bool {
+        return (cs.c != 0 || ctl.wait(bar(S::kBQ + (cs.xi & 1)), uint32_t(cs.xi >> 1) & 1u)) &&
+               ctl.wait(bar(S::kBK + (cs.g & 1)), uint32_t(cs.g >> 1) & 1u);
+      };
+      // S of step s (cursor cs) into the S buffer
+      auto issue_s = [&](const DqCursor& cs) {
         tc_fence_after();
         const uint32_t qb = sQ(cs.xi & 1), kb = sK(cs.g);
 #pragma unroll
@@ -435,11 +439,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + S::kColS, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
         }
         tc_commit(bar(S::kBS));
-        return true;
       };
-      // dP of step s into the dP buffer, once its V has landed
-      auto issue_dp = [&](const DqCursor& cs) -> bool {
-        if (!ctl.wait(bar(S::kBV), uint32_t(cs.g) & 1u)) return false;
+      // dP of step s into the dP buffer
+      auto issue_dp = [&](const DqCursor& cs) {
         tc_fence_after();
         const uint32_t qb = sQ(cs.xi & 1) + S::kQBytes;
 #pragma unroll
@@ -449,11 +451,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(S::kBDP));
         if (cs.c == dq_steps(cs.it) - 1) tc_commit(bar(S::kBQFree + (cs.xi & 1)));   // last reader of Q, dO
-        return true;
       };
       DqCursor cd{0, 0, 0, 0, {}, false};
       seek(cd, true);
-      if (cd.valid) ok = issue_s(cd) && issue_dp(cd);
+      if (cd.valid) {
+        ok = loads_s(cd) && ctl.wait(bar(S::kBV), uint32_t(cd.g) & 1u);
+        if (ok) {
+          issue_s(cd);
+          issue_dp(cd);
+        }
+      }
       while (ok && cd.valid) {
         DqCursor nx = cd;                      // the next step (same item or the next one)
         {
@@ -465,15 +472,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             seek(nx, false);
           }
         }
+        if (nx.valid && !(ok = loads_s(nx))) break;
         // the row threads have read S(s) and dP(s): S(s + 1) may overwrite S
         if (!(ok = ctl.wait(bar(S::kBRead), uint32_t(cd.g) & 1u))) break;
-        if (nx.valid && !(ok = issue_s(nx))) break;
+        if (nx.valid) issue_s(nx);
         // dQ(s) once dS(s) is in TMEM (and, for a tile's first step, its
-        // accumulator has been read out for the tile two before)
-        if (!(ok = ctl.wait(bar(S::kBDS), uint32_t(cd.g) & 1u))) break;
+        // accumulator has been read out for the tile two before); dP(s + 1)
+        // overwrites the dP buffer after dQ(s) has read it (same queue)
+        if (nx.valid && !(ok = ctl.wait(bar(S::kBV), uint32_t(nx.g) & 1u))) break;
         if (cd.c == 0 && cd.xi >= 2 &&
             !(ok = ctl.wait(bar(S::kBAccFree + (cd.xi & 1)), uint32_t((cd.xi - 2) >> 1) & 1u)))
           break;
+        if (!(ok = ctl.wait(bar(S::kBDS), uint32_t(cd.g) & 1u))) break;
         tc_fence_after();
         {
           const uint32_t kb = sK(cd.g);
@@ -486,8 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bar(S::kBKFree + (cd.g & 1)));
           if (cd.c == dq_steps(cd.it) - 1) tc_commit(bar(S::kBAcc + (cd.xi & 1)));
         }
-        // dP(s + 1) overwrites the dP buffer after dQ(s) has read it (same queue)
-        if (nx.valid && !(ok = issue_dp(nx))) break;
+        if (nx.valid) issue_dp(nx);
         advance(cd, true);
       }
       tc_commit(bar(S::kBDrain));
