@@ -822,25 +822,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       Idle idle;
       while (cd.valid && ok) {
         bool progress = false;
-        // S(t), dP(t): TMEM buffer t & 1 is free once tile t - 2's dV / dK are issued
-        if (cs.valid && cs.t < cd.t + 2 &&
-            (cs.e > 0 || mbar_test(bar(S::kBKV + (cs.y & 1)), uint32_t(cs.y >> 1) & 1u)) &&
-            mbar_test(bar(S::kBQ + (cs.t & 1)), uint32_t(cs.t >> 1) & 1u)) {
-          tc_fence_after();
-          const uint32_t qb = sQ(cs.t), kb = sKV(cs.y), vb = kb + S::kTile;
-          const uint32_t ds = tmem + S::kColS + (cs.t & 1) * kChunk, ddp = tmem + S::kColDP + (cs.t & 1) * kChunk;
-#pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
-            mma_ss(ds, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
-            mma_ss(ddp, sw128_desc(qb + S::kQBytes + ao, 16, 1024), sw128_desc(vb + bo, 16, 1024), S::kIdescS,
-                   kk > 0);
-          }
-          tc_commit(bar(S::kBS + (cs.t & 1)));
-          if (cs.e == cs.it.total - 1) tc_commit(bar(S::kBKVFree + (cs.y & 1)));
-          advance(cs, false);
-          progress = true;
-        }
         // dV^T += dO^T P, dK^T += Q^T dS for tile t, once its P / dS are written
         if ((cd.t < cs.t || !cs.valid) && mbar_test(bar(S::kBPDS), uint32_t(cd.t) & 1u) &&
             (cd.e > 0 || cd.y < 2 ||
@@ -860,6 +841,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit(bar(S::kBDone + (cd.t & 1)));
           if (cd.e == cd.it.total - 1) tc_commit(bar(S::kBAcc + (cd.y & 1)));
           advance(cd, true);
+          progress = true;
+        }
+        // S(t), dP(t): TMEM buffer t & 1 is free once tile t - 2's dV / dK are issued
+        if (cs.valid && cs.t < cd.t + 2 &&
+            (cs.e > 0 || mbar_test(bar(S::kBKV + (cs.y & 1)), uint32_t(cs.y >> 1) & 1u)) &&
+            mbar_test(bar(S::kBQ + (cs.t & 1)), uint32_t(cs.t >> 1) & 1u)) {
+          tc_fence_after();
+          const uint32_t qb = sQ(cs.t), kb = sKV(cs.y), vb = kb + S::kTile;
+          const uint32_t ds = tmem + S::kColS + (cs.t & 1) * kChunk, ddp = tmem + S::kColDP + (cs.t & 1) * kChunk;
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
+            mma_ss(ds, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
+            mma_ss(ddp, sw128_desc(qb + S::kQBytes + ao, 16, 1024), sw128_desc(vb + bo, 16, 1024), S::kIdescS,
+                   kk > 0);
+          }
+          tc_commit(bar(S::kBS + (cs.t & 1)));
+          if (cs.e == cs.it.total - 1) tc_commit(bar(S::kBKVFree + (cs.y & 1)));
+          advance(cs, false);
           progress = true;
         }
         ok = ok && idle.step(progress, ctl);
