@@ -315,11 +315,12 @@ def main():
     ap.add_argument("--only-device", action="store_true",
                     help="device-timed leg only (no e2e, CPU baseline or other workloads); "
                          "the form used for profiler captures")
-    ap.add_argument("--leg", default=None, choices=["backward", "bsbr"],
-                    help="time one secondary leg alone on --workload (backward) or the BSBR "
-                         "workload (bsbr) and print its JSON; the form used for profiler captures")
+    ap.add_argument("--leg", default=None, choices=["backward", "bsbr", "decode"],
+                    help="time one secondary leg alone on --workload (backward), the BSBR "
+                         "workload (bsbr) or the headline route's decode (decode) and print its "
+                         "JSON; the form used for profiler captures")
     ap.add_argument("--n", type=int, default=None,
-                    help="with --leg backward: the workload's geometry at this sequence length "
+                    help="with --leg backward or decode: the workload's geometry at this sequence length "
                          "(a smaller case for full profiler captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -547,6 +548,8 @@ def run_leg(args, w):
         if args.n is not None:
             w = dataclasses.replace(w, n=args.n)
         res = bench_backward(w, dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup)
+    elif args.leg == "decode":
+        res = bench_decode(dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup, n=args.n)
     else:
         w = WORKLOADS["bsbr_block_diagonal"]
         res = bench_bsbr(w, dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup)
@@ -685,12 +688,15 @@ def bench_bsbr(w, dev, stream, flush, bsa, torch, steps=20, warmup=3):
     return res
 
 
-def bench_decode(dev, stream, flush, bsa, torch, batches=(1, 32), steps=20, warmup=3):
+def bench_decode(dev, stream, flush, bsa, torch, batches=(1, 32), steps=20, warmup=3, n=None):
     """Selected-page decode on the headline route: each sequence's new token at
     the last position of a 32K context, reading its block row's kept pages
     through a shuffled page table.  Reports time per step and the unique
     key/value bytes of the kept pages (what a step must read) per second."""
+    import dataclasses
     w = WORKLOADS[HEADLINE]
+    if n is not None:
+        w = dataclasses.replace(w, n=n)
     lay = bsa.Layout.for_workload(w, dev)
     row_ptr, col_idx = lay.csr()
     H, hkv, B, d, n = w.q_heads, w.kv_heads_per_seq, w.B, w.d, w.n

@@ -7,25 +7,31 @@
 //
 // A query row is a single vector, so the step is a stream over the kept
 // pages' keys and values (HBM/L2 bound, no matrix product to hand to the
-// tensor cores).  One CTA serves two query rows of a key/value head's group
-// when they share a route (one layout head, an even group), else one row, so
-// a group's rows read each kept page once.  Its 16 warps take the kept blocks in turn.  For a
-// block, 8 lanes cooperate on each key row (16-byte loads, the row read as
-// one coalesced line; a 3-step shuffle tree sums the dot product), four rows
-// per step, scoring the row against all G queries held in shared memory; the
-// scores go through shared memory for the block's max, exponentials and sum
-// (an fp32 online softmax per query), and P V is accumulated with lanes across
-// d.  The warps' partial (max, sum, o) are then merged in shared memory.
-// Everything is fp32 (P is not rounded to bf16); o is stored as bf16 and lse
-// in fp32.
+// tensor cores).  The unit of work is a task: 32 consecutive key rows of one
+// kept page, i.e. one contiguous K run and one contiguous V run of the page's
+// tile for the key/value head.  A thread-block cluster of C CTAs (C = 1..8,
+// chosen on the host from the layout's longest row and the number of query
+// groups, so that short rows spread over many SMs and long batches do not
+// oversubscribe them) serves G query rows of one key/value head (G = 2 when
+// two rows of a group share a route, else 1); the row's tasks are dealt
+// round-robin over the cluster's warps.  Each warp double-buffers its tasks
+// (two bulk copies per task on one mbarrier, the next task's copies issued
+// before the current one is scored), with the page numbers of 32 tasks
+// fetched at once by its lanes.  Scoring: 8 lanes per key row, four rows per
+// step, q held in registers, packed fp32 FMAs; a warp keeps an fp32 online
+// softmax per query (P is not rounded to bf16) and accumulates P V with lanes
+// across d.  The warps' partial (max, sum, o) are merged in shared memory,
+// then the cluster's CTAs' partials are merged by CTA 0 through distributed
+// shared memory; o is stored as bf16 and lse in fp32.
 //
 // Positions and page numbers come from device memory: a position outside
 // [0, n) or a page outside [0, num_pages) is not read; the kernel records a
 // status bit (reported by bsa_get_status) and writes o = 0, lse = -inf for
-// the rows of that CTA.
+// the rows of that cluster.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 #include <string>
@@ -35,9 +41,11 @@
 namespace bsa {
 namespace dec {
 
-constexpr int kTileBudget = 192 * 1024;   // shared memory for the warps' K/V tiles
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // a copy that takes longer than 1 s is abandoned
+constexpr int kRows = 32;                           // key rows per task
+constexpr int kMaxCluster = 8;                      // portable cluster size
+constexpr uint64_t kWaitLimitNs = 1000000000ull;    // a copy that takes longer than 1 s is abandoned
 constexpr float kLn2 = 0.693147180559945309f;
+constexpr int kFlagBadIndex = 1, kFlagTimeout = 2;
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -52,8 +60,20 @@ struct DecodeParams {
   uint32_t* status;
   int n, nb, L, max_blocks, num_pages;
   int H, hkv, g;        // query heads and key/value heads per sequence, H / hkv
+  int C;                // CTAs per cluster (the grid's x extent is query groups * C)
   float scale_log2;
 };
+
+// Warps per CTA: two buffers of a task's K and V tiles per warp, 96 KB of
+// tiles per CTA, so two CTAs fit one SM.
+template <int HD>
+__host__ __device__ constexpr int warps_per_cta() {
+  return HD == 128 ? 3 : 6;
+}
+template <int HD>
+__host__ __device__ constexpr uint32_t task_tile_bytes() {   // one task's K (or V) rows
+  return uint32_t(kRows) * HD * 2;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -63,7 +83,7 @@ __device__ __forceinline__ uint64_t gtimer() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// One contiguous tile global -> shared by the bulk-copy engine (no multicast),
+// One contiguous run global -> shared by the bulk-copy engine (no multicast),
 // completing the given mbarrier's transaction count.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -84,53 +104,119 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
     if (gtimer() - t0 > kWaitLimitNs) return false;
   }
 }
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-// G query rows per CTA (2 when the rows of a group share a route, else 1).
-template <int BLK, int HD>
-__host__ __device__ constexpr int warps_for() {   // as many warps as K and V tiles of a page fit the budget, at most 6
-  return kTileBudget / (2 * BLK * HD * 2) < 6 ? kTileBudget / (2 * BLK * HD * 2) : 6;
+// (d0, d1) += (a0, a1) * (b0, b1), two fp32 lanes in one instruction, each
+// rounded as the scalar fma would be.
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rd, {%0, %1};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rd;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// bf16 pair (low half first) to two floats: a bf16 is the high half of an fp32.
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
+  lo = __uint_as_float(w << 16);
+  hi = __uint_as_float(w & 0xffff0000u);
+}
+__device__ __forceinline__ int cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return int(r);
+}
+// Every thread of every CTA of the cluster: writes before are visible to the
+// cluster's reads after.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, int rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ float ld_peer_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+__device__ __forceinline__ int ld_peer_s32(uint32_t a) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+  return v;
 }
 
 template <int BLK, int HD, int G>
-__global__ void __launch_bounds__(warps_for<BLK, HD>() * 32) bsa_decode_kernel(const DecodeParams p) {
-  constexpr int kWarps = warps_for<BLK, HD>();
+__global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(const DecodeParams p) {
+  constexpr int W = warps_per_cta<HD>();
+  constexpr int PB = BLK / kRows;     // tasks per page
   constexpr int CPL = HD / 8;         // key columns per lane (8 lanes per key row)
   constexpr int DPL = HD / 32;        // o columns per lane
-  constexpr uint32_t kTile = BLK * HD * 2;   // one page's K (or V) tile of one head
-  extern __shared__ __align__(128) uint8_t dyn[];   // per warp: K tile, V tile
-  __shared__ __align__(8) uint64_t tile_bar[kWarps];
-  __shared__ float sq[G][HD];
-  __shared__ float sp[kWarps][G][BLK];          // scores, then P, of a warp's block
-  __shared__ float sm[kWarps][G], sl[kWarps][G];
-  __shared__ float so[kWarps][G][HD];
-  __shared__ int s_bad;
-  // the CTA's rows f0 .. f0 + G - 1 (G divides g, so they share a key/value head)
-  const int f0 = blockIdx.x * G;
+  constexpr uint32_t kTile = task_tile_bytes<HD>();
+  constexpr unsigned kAll = 0xffffffffu;
+  extern __shared__ __align__(128) uint8_t dyn[];   // per warp: 2 x (K tile, V tile)
+  __shared__ __align__(8) uint64_t bars[W][2];
+  __shared__ float sp[W][G][kRows];               // scores, then P, of a warp's task
+  __shared__ float sm[W][G], sl[W][G];
+  __shared__ float so[W][G][HD];
+  __shared__ float cm[G], cl[G];                  // the CTA's merged partial state
+  __shared__ float co[G][HD];
+  __shared__ int s_flags, s_start, s_len, s_t;
+
+  const int C = p.C;
+  const int rank = cluster_rank();
+  const int f0 = (blockIdx.x / C) * G;            // the cluster's rows f0 .. f0 + G - 1
   const int b = f0 / p.H;
   const int hk = (f0 - b * p.H) / p.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float sl2 = p.scale_log2;
-  for (int c = threadIdx.x; c < G * HD; c += blockDim.x)
-    sq[c / HD][c % HD] = __bfloat162float(p.q[size_t(f0) * HD + c]);
-  if (threadIdx.x == 0) s_bad = 0;
+  if (threadIdx.x == 0) {
+    const int t = p.positions[b];
+    int start = 0, len = 0, flags = 0;
+    if (t >= 0 && t < p.n) {
+      const size_t row = size_t(f0 % p.L) * p.nb + t / BLK;
+      start = p.row_ptr[row];
+      len = p.row_ptr[row + 1] - start;
+    } else {
+      flags = kFlagBadIndex;
+    }
+    s_t = t;
+    s_start = start;
+    s_len = len;
+    s_flags = flags;
+  }
   if (lane == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&tile_bar[warp])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp][0])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp][1])) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  // this lane's query columns, in registers
+  const int sub = lane >> 3, pc = lane & 7;       // key row within a step of 4, column slice
+  float qr[G][CPL];
+#pragma unroll
+  for (int gq = 0; gq < G; ++gq) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + size_t(f0 + gq) * HD + pc * CPL);
+#pragma unroll
+    for (int c8 = 0; c8 < CPL / 8; ++c8) {
+      const uint4 w = src[c8];
+      bf16x2_to_f32(w.x, qr[gq][c8 * 8 + 0], qr[gq][c8 * 8 + 1]);
+      bf16x2_to_f32(w.y, qr[gq][c8 * 8 + 2], qr[gq][c8 * 8 + 3]);
+      bf16x2_to_f32(w.z, qr[gq][c8 * 8 + 4], qr[gq][c8 * 8 + 5]);
+      bf16x2_to_f32(w.w, qr[gq][c8 * 8 + 6], qr[gq][c8 * 8 + 7]);
+    }
+  }
   __syncthreads();
-  const uint32_t bar = smem_u32(&tile_bar[warp]);
-  const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(dyn + size_t(warp) * 2 * kTile);
-  const __nv_bfloat16* vt = kt + BLK * HD;
-  int loads = 0;                      // tiles pairs this warp has brought in (barrier phases)
 
-  const int t = p.positions[b];
-  const bool pos_ok = t >= 0 && t < p.n;
+  const int t = s_t, start = s_start, len = s_len;
+  const int T = len * PB;                         // tasks of the row
+  const int gw = rank * W + warp, S = C * W;      // this warp's first task, stride
+  const int mine = T > gw ? (T - gw + S - 1) / S : 0;
+  uint8_t* wbase = dyn + size_t(warp) * 4 * kTile;
+  const uint32_t bar0 = smem_u32(&bars[warp][0]);
   float m[G], l[G], acc[G][DPL];
 #pragma unroll
   for (int gq = 0; gq < G; ++gq) {
@@ -139,133 +225,148 @@ __global__ void __launch_bounds__(warps_for<BLK, HD>() * 32) bsa_decode_kernel(c
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[gq][e] = 0.f;
   }
-  if (pos_ok) {
-    const int i = t / BLK;
-    const size_t row = size_t(f0 % p.L) * p.nb + i;
-    const int start = p.row_ptr[row], len = p.row_ptr[row + 1] - start;
-    const int sub = lane >> 3, part = lane & 7;   // key row within a step of 4, column slice
-    for (int e = warp; e < len; e += kWarps) {
-      const int j = p.col_idx[start + e];
-      const int page = p.page_table[size_t(b) * p.max_blocks + j];
-      if (page < 0 || page >= p.num_pages) {
-        if (lane == 0) s_bad = 1;
-        continue;
+  // lane x holds the key block and page of local task m0 + x
+  int m0 = -kRows, idx_j = 0, idx_page = -1;
+  // per buffer: first key of the task in it; bit k of `live`: copies in flight into buffer k
+  int u_first0 = 0, u_first1 = 0;
+  uint32_t live = 0;
+  uint32_t phase = 0;                             // bit k: parity of buffer k's next completion
+  int flags = 0;
+
+  // Issue the copies of local task mt into buffer mt & 1 (nothing for a task
+  // past the token or with a refused page).
+  auto issue = [&](int mt) {
+    if (mt - m0 >= 32) {
+      m0 = mt;
+      const int x = mt + lane;
+      idx_j = 0;
+      idx_page = -1;
+      if (x < mine) {
+        const int k = gw + x * S;
+        idx_j = p.col_idx[start + k / PB];
+        idx_page = p.page_table[size_t(b) * p.max_blocks + idx_j];
       }
-      const size_t tile = (size_t(page) * p.hkv + hk) * BLK * HD;
-      // this block's K and V tiles into the warp's buffers, one bulk copy each
-      __syncwarp();                      // every lane is done with the previous tiles
-      if (lane == 0) {
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads before the copy
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTile)
-                     : "memory");
-        bulk_load(smem_u32(kt), p.kc + tile, kTile, bar);
-        bulk_load(smem_u32(vt), p.vc + tile, kTile, bar);
-      }
-      const bool landed = bar_wait(bar, uint32_t(loads) & 1u);
-      ++loads;
-      if (!__all_sync(0xffffffffu, landed)) {
-        if (lane == 0) s_bad = 2;
-        break;
-      }
-      // ---- scores: rows 4 * step + sub, columns part * CPL ..
-#pragma unroll 4
-      for (int step = 0; step < BLK / 4; ++step) {
-        const int r = step * 4 + sub;
-        const uint4* kr = reinterpret_cast<const uint4*>(kt + size_t(r) * HD + part * CPL);
-        float dot[G];
+    }
+    const int j = __shfl_sync(kAll, idx_j, mt - m0);
+    const int page = __shfl_sync(kAll, idx_page, mt - m0);
+    const int part = (gw + mt * S) % PB;
+    const int bi = mt & 1;
+    const int u_first = j * BLK + part * kRows;
+    if (bi) u_first1 = u_first; else u_first0 = u_first;
+    if (page < 0 || page >= p.num_pages) {
+      flags |= kFlagBadIndex;
+      return;
+    }
+    if (u_first > t) return;                       // every key of the task is after the token
+    live |= 1u << bi;
+    __syncwarp();                                  // every lane is done with the buffer's last task
+    if (lane == 0) {
+      const uint32_t bar = bar0 + 8u * bi;
+      const size_t off = ((size_t(page) * p.hkv + hk) * BLK + size_t(part) * kRows) * HD;
+      uint8_t* kt = wbase + size_t(bi) * 2 * kTile;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads before the copy
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTile) : "memory");
+      bulk_load(smem_u32(kt), p.kc + off, kTile, bar);
+      bulk_load(smem_u32(kt + kTile), p.vc + off, kTile, bar);
+    }
+  };
+
+  if (mine > 0) issue(0);
+  for (int mt = 0; mt < mine; ++mt) {
+    const int bi = mt & 1;
+    if (mt + 1 < mine) issue(mt + 1);
+    if (!((live >> bi) & 1u)) continue;
+    const bool landed = bar_wait(bar0 + 8u * bi, (phase >> bi) & 1u);
+    phase ^= 1u << bi;
+    live &= ~(1u << bi);
+    if (!__all_sync(kAll, landed)) {
+      flags |= kFlagTimeout;
+      break;
+    }
+    const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(wbase + size_t(bi) * 2 * kTile);
+    const __nv_bfloat16* vt = kt + kRows * HD;
+    const int u0 = bi ? u_first1 : u_first0;       // the task's first key
+    // ---- scores: rows 4 * step + sub, columns pc * CPL ..
+#pragma unroll 2
+    for (int step = 0; step < kRows / 4; ++step) {
+      const int r = step * 4 + sub;
+      const uint4* kr = reinterpret_cast<const uint4*>(kt + size_t(r) * HD + pc * CPL);
+      float d0[G], d1[G];
 #pragma unroll
-        for (int gq = 0; gq < G; ++gq) dot[gq] = 0.f;
+      for (int gq = 0; gq < G; ++gq) d0[gq] = d1[gq] = 0.f;
 #pragma unroll
-        for (int c8 = 0; c8 < CPL / 8; ++c8) {
-          const uint4 w = kr[c8];
-          const __nv_bfloat162* pr = reinterpret_cast<const __nv_bfloat162*>(&w);
+      for (int c8 = 0; c8 < CPL / 8; ++c8) {
+        const uint4 w = kr[c8];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const float2 kv = __bfloat1622float2(pr[e2]);
-            const int c = part * CPL + c8 * 8 + 2 * e2;
+        for (int e2 = 0; e2 < 4; ++e2) {
+          float k0, k1;
+          bf16x2_to_f32(ws[e2], k0, k1);
 #pragma unroll
-            for (int gq = 0; gq < G; ++gq) {
-              dot[gq] = fmaf(kv.x, sq[gq][c], dot[gq]);
-              dot[gq] = fmaf(kv.y, sq[gq][c + 1], dot[gq]);
-            }
-          }
+          for (int gq = 0; gq < G; ++gq)
+            fma2(d0[gq], d1[gq], k0, k1, qr[gq][c8 * 8 + 2 * e2], qr[gq][c8 * 8 + 2 * e2 + 1]);
         }
-#pragma unroll
-        for (int gq = 0; gq < G; ++gq) {
-          dot[gq] += __shfl_xor_sync(0xffffffffu, dot[gq], 1);
-          dot[gq] += __shfl_xor_sync(0xffffffffu, dot[gq], 2);
-          dot[gq] += __shfl_xor_sync(0xffffffffu, dot[gq], 4);
-        }
-        if (part == 0) {
-          const bool allowed = j * BLK + r <= t;   // causal; other blocks of the route are earlier
-#pragma unroll
-          for (int gq = 0; gq < G; ++gq) sp[warp][gq][r] = allowed ? dot[gq] * sl2 : -INFINITY;
-        }
       }
-      __syncwarp();
-      // ---- online softmax per query over this block's keys
-      float alpha[G];
-      bool any = false;
 #pragma unroll
       for (int gq = 0; gq < G; ++gq) {
-        float bm = -INFINITY;
-#pragma unroll
-        for (int r = lane; r < BLK; r += 32) bm = fmaxf(bm, sp[warp][gq][r]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
-        const float m_new = fmaxf(m[gq], bm);
-        alpha[gq] = (m_new == -INFINITY) ? 1.f : ex2(m[gq] - m_new);   // 0 when m was -inf
-        float psum = 0.f;
-#pragma unroll
-        for (int r = lane; r < BLK; r += 32) {
-          const float pv = (m_new == -INFINITY) ? 0.f : ex2(sp[warp][gq][r] - m_new);
-          sp[warp][gq][r] = pv;
-          psum += pv;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
-        l[gq] = l[gq] * alpha[gq] + psum;
-        m[gq] = m_new;
-        any = any || bm != -INFINITY;
+        float dot = d0[gq] + d1[gq];
+        dot += __shfl_xor_sync(kAll, dot, 1);
+        dot += __shfl_xor_sync(kAll, dot, 2);
+        dot += __shfl_xor_sync(kAll, dot, 4);
+        if (pc == 0) sp[warp][gq][r] = (u0 + r <= t) ? dot * sl2 : -INFINITY;
       }
-      __syncwarp();
-      if (!any) continue;                        // nothing allowed in this block
-      // ---- O += P V: lane owns columns lane * DPL ..
-#pragma unroll
-      for (int gq = 0; gq < G; ++gq)
-#pragma unroll
-        for (int e2 = 0; e2 < DPL; ++e2) acc[gq][e2] *= alpha[gq];
-#pragma unroll 8
-      for (int r = 0; r < BLK; ++r) {
-        const __nv_bfloat16* vr = vt + size_t(r) * HD + lane * DPL;
-        float vv[DPL];
-        if constexpr (DPL == 4) {
-          const uint2 w = *reinterpret_cast<const uint2*>(vr);
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.x));
-          const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w.y));
-          vv[0] = a.x;
-          vv[1] = a.y;
-          vv[2] = c.x;
-          vv[3] = c.y;
-        } else {
-          const uint32_t w = *reinterpret_cast<const unsigned int*>(vr);
-          const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w));
-          vv[0] = a.x;
-          vv[1] = a.y;
-        }
-#pragma unroll
-        for (int gq = 0; gq < G; ++gq) {
-          const float pu = sp[warp][gq][r];
-#pragma unroll
-          for (int e2 = 0; e2 < DPL; ++e2) acc[gq][e2] = fmaf(pu, vv[e2], acc[gq][e2]);
-        }
-      }
-      __syncwarp();
     }
-  } else if (threadIdx.x == 0) {
-    s_bad = 1;
+    __syncwarp();
+    // ---- online softmax per query; lane x owns key row x of the task
+#pragma unroll
+    for (int gq = 0; gq < G; ++gq) {
+      const float s = sp[warp][gq][lane];
+      float bm = s;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(kAll, bm, off));
+      const float m_new = fmaxf(m[gq], bm);        // finite: the task's first key is allowed
+      const float alpha = ex2(m[gq] - m_new);      // 0 while m is -inf
+      const float pv = ex2(s - m_new);             // 0 for a disallowed key
+      sp[warp][gq][lane] = pv;
+      float psum = pv;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(kAll, psum, off);
+      l[gq] = l[gq] * alpha + psum;
+      m[gq] = m_new;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[gq][e] *= alpha;
+    }
+    __syncwarp();
+    // ---- O += P V: lane owns columns lane * DPL ..
+#pragma unroll 8
+    for (int r = 0; r < kRows; ++r) {
+      const __nv_bfloat16* vr = vt + size_t(r) * HD + lane * DPL;
+      float vv[DPL];
+      if constexpr (DPL == 4) {
+        const uint2 w = *reinterpret_cast<const uint2*>(vr);
+        bf16x2_to_f32(w.x, vv[0], vv[1]);
+        bf16x2_to_f32(w.y, vv[2], vv[3]);
+      } else {
+        bf16x2_to_f32(*reinterpret_cast<const uint32_t*>(vr), vv[0], vv[1]);
+      }
+#pragma unroll
+      for (int gq = 0; gq < G; ++gq) {
+        const float pu = sp[warp][gq][r];
+#pragma unroll
+        for (int e2 = 0; e2 < DPL; e2 += 2) fma2(acc[gq][e2], acc[gq][e2 + 1], pu, pu, vv[e2], vv[e2 + 1]);
+      }
+    }
+    __syncwarp();
   }
-  // merge the warps' partial softmax states
+  // leave no copy in flight into shared memory
+  if (lane == 0) {
+#pragma unroll
+    for (int bi = 0; bi < 2; ++bi)
+      if (((live >> bi) & 1u) && !bar_wait(bar0 + 8u * bi, (phase >> bi) & 1u)) flags |= kFlagTimeout;
+  }
+  flags = __reduce_or_sync(kAll, flags);
+  if (lane == 0 && flags) atomicOr(&s_flags, flags);
+  // ---- merge the warps' partial softmax states
 #pragma unroll
   for (int gq = 0; gq < G; ++gq) {
     if (lane == 0) {
@@ -273,64 +374,110 @@ __global__ void __launch_bounds__(warps_for<BLK, HD>() * 32) bsa_decode_kernel(c
       sl[warp][gq] = l[gq];
     }
 #pragma unroll
-    for (int e2 = 0; e2 < DPL; ++e2) so[warp][gq][lane * DPL + e2] = acc[gq][e2];
+    for (int e = 0; e < DPL; ++e) so[warp][gq][lane * DPL + e] = acc[gq][e];
   }
   __syncthreads();
-  // a refused index (or a copy that never landed): the CTA's rows are o = 0,
-  // lse = -inf.  Leave no copy in flight into shared memory.
-  if (lane == 0 && loads > 0) bar_wait(bar, uint32_t(loads - 1) & 1u);
-  __syncwarp();
-  const bool bad = s_bad != 0;
-  for (int c = threadIdx.x; c < G * HD; c += blockDim.x) {
+  for (int c = threadIdx.x; c < G * HD; c += W * 32) {
     const int gq = c / HD, col = c % HD;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sm[w][gq]);
+    for (int w = 0; w < W; ++w) M = fmaxf(M, sm[w][gq]);
     float Lsum = 0.f, v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < W; ++w) {
       const float wt = (M == -INFINITY) ? 0.f : ex2(sm[w][gq] - M);
       Lsum += wt * sl[w][gq];
       v += wt * so[w][gq][col];
     }
-    const bool ok = Lsum > 0.f && !bad;
-    p.o[size_t(f0 + gq) * HD + col] = __float2bfloat16_rn(ok ? v / Lsum : 0.f);
-    if (col == 0) p.lse[f0 + gq] = ok ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+    co[gq][col] = v;
+    if (col == 0) {
+      cm[gq] = M;
+      cl[gq] = Lsum;
+    }
   }
-  if (threadIdx.x == 0 && bad) atomicOr(p.status, s_bad == 2 ? kStatusTimeout : kStatusBadIndex);
+  // ---- merge the cluster's CTAs (CTA 0 reads the others' shared memory)
+  cluster_sync();
+  if (rank == 0) {
+    int all_flags = 0;
+    for (int r = 0; r < C; ++r) all_flags |= ld_peer_s32(peer_addr(&s_flags, r));
+    for (int c = threadIdx.x; c < G * HD; c += W * 32) {
+      const int gq = c / HD, col = c % HD;
+      float M = -INFINITY;
+      for (int r = 0; r < C; ++r) M = fmaxf(M, ld_peer_f32(peer_addr(&cm[gq], r)));
+      float Lsum = 0.f, v = 0.f;
+      for (int r = 0; r < C; ++r) {
+        const float wt = (M == -INFINITY) ? 0.f : ex2(ld_peer_f32(peer_addr(&cm[gq], r)) - M);
+        Lsum += wt * ld_peer_f32(peer_addr(&cl[gq], r));
+        v += wt * ld_peer_f32(peer_addr(&co[gq][col], r));
+      }
+      const bool ok = Lsum > 0.f && all_flags == 0;
+      p.o[size_t(f0 + gq) * HD + col] = __float2bfloat16_rn(ok ? v / Lsum : 0.f);
+      if (col == 0) p.lse[f0 + gq] = ok ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+    }
+    if (threadIdx.x == 0 && all_flags)
+      atomicOr(p.status, (all_flags & kFlagTimeout ? kStatusTimeout : 0u) |
+                             (all_flags & kFlagBadIndex ? kStatusBadIndex : 0u));
+  }
+  cluster_sync();                                   // CTA 0 is done reading the others
+}
+
+// CTAs per cluster: enough warps for one task each on the longest row, cut
+// back while the grid would exceed the CTAs the GPU holds at once.
+inline int cluster_size(int groups, int max_row, int tasks_per_page, int warps, int resident) {
+  const int tasks = std::max(1, max_row * tasks_per_page);
+  int c = std::min(kMaxCluster, (tasks + warps - 1) / warps);
+  while (c > 1 && size_t(groups) * c > size_t(resident)) c = (c + 1) / 2;
+  return std::max(c, 1);
 }
 
 template <int BLK, int HD, int G>
-int launch_g(const DecodeParams& p, int heads, cudaStream_t s) {
+int launch_g(DecodeParams p, int heads, int max_row, cudaStream_t s) {
   auto kern = bsa_decode_kernel<BLK, HD, G>;
-  constexpr int kWarps = warps_for<BLK, HD>();
-  const int smem = kWarps * 2 * BLK * HD * 2;
+  constexpr int W = warps_per_cta<HD>();
+  const int smem = W * 4 * int(task_tile_bytes<HD>());
   // the attribute is a property of the function: set it once per device
   static std::mutex mu;
   static bool done[64] = {};
+  static int sms[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) return set_error(BSA_ERR_CUDA, "cannot query the device");
+  int n_sm = 0;
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!done[dev]) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode smem: ") + cudaGetErrorString(e));
+      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode SMs: ") + cudaGetErrorString(e));
       done[dev] = true;
     }
+    n_sm = sms[dev];
   }
-  kern<<<heads / G, kWarps * 32, smem, s>>>(p);
+  const int groups = heads / G;
+  p.C = cluster_size(groups, max_row, BLK / kRows, W, 2 * n_sm);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(groups * p.C), 1, 1);
+  cfg.blockDim = dim3(W * 32, 1, 1);
+  cfg.dynamicSmemBytes = size_t(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = unsigned(p.C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, p);
+  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
   return BSA_OK;
 }
 
 template <int BLK, int HD>
-int launch(const DecodeParams& p, int heads, cudaStream_t s) {
-  // two query rows of a key/value head's group per CTA when they share a route
-  const int st = (p.L == 1 && p.g % 2 == 0) ? launch_g<BLK, HD, 2>(p, heads, s) : launch_g<BLK, HD, 1>(p, heads, s);
-  if (st != BSA_OK) return st;
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
-  return BSA_OK;
+int launch(const DecodeParams& p, int heads, int max_row, cudaStream_t s) {
+  // two query rows of a key/value head's group per cluster when they share a route
+  return (p.L == 1 && p.g % 2 == 0) ? launch_g<BLK, HD, 2>(p, heads, max_row, s)
+                                    : launch_g<BLK, HD, 1>(p, heads, max_row, s);
 }
 
 }  // namespace dec
@@ -388,8 +535,9 @@ extern "C" int bsa_decode(const void* q, const void* k_cache, const void* v_cach
   p.g = H / hkv;
   p.scale_log2 = float(double(scale) * 1.4426950408889634);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (B == 64 && d == 128) return dec::launch<64, 128>(p, heads, s);
-  if (B == 64 && d == 64) return dec::launch<64, 64>(p, heads, s);
-  if (B == 128 && d == 128) return dec::launch<128, 128>(p, heads, s);
-  return dec::launch<128, 64>(p, heads, s);
+  const int mr = layout->max_row;
+  if (B == 64 && d == 128) return dec::launch<64, 128>(p, heads, mr, s);
+  if (B == 64 && d == 64) return dec::launch<64, 64>(p, heads, mr, s);
+  if (B == 128 && d == 128) return dec::launch<128, 128>(p, heads, mr, s);
+  return dec::launch<128, 64>(p, heads, mr, s);
 }

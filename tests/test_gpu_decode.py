@@ -86,6 +86,22 @@ def test_decode_full_32k_dyadic():
     lay.close()
 
 
+def test_decode_long_rows_many_tasks_per_warp():
+    """Full causal rows of up to 512 pages: each warp of a cluster takes more
+    than 32 tasks of 32 key rows, so its page numbers are fetched in several
+    rounds; positions 31 and 32 put the token at the end of a task and at the
+    first key of the next one."""
+    n, B, batch, H, hkv, d = 32768, 64, 1, 2, 1, 128
+    nb = n // B
+    lay, sets, dev_t, host = _setup(OL.BAND_GLOBAL, n, B, 1, batch, H, hkv, d,
+                                    dict(window=nb, global_first=0), seed=7)
+    for positions in ([n - 1], [n // 2 + 5], [31], [32]):
+        o, lse, o_ref, lse_ref = _step(lay, sets, dev_t, host, batch, H, d, B, positions, 1.0 / math.sqrt(d))
+        assert_close(o, lse, o_ref, lse_ref, f"decode full causal rows, positions {positions}")
+    bsa.bsa_get_status(lay.handle)
+    lay.close()
+
+
 def test_decode_refuses_bad_indices_on_device():
     n, B, batch, H, hkv, d = 1024, 64, 2, 2, 2, 64
     lay, sets, dev_t, host = _setup(OL.DYADIC, n, B, 1, batch, H, hkv, d,
