@@ -549,6 +549,8 @@ def run_leg(args, w):
             w = dataclasses.replace(w, n=args.n)
         res = bench_backward(w, dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup)
     elif args.leg == "decode":
+        if args.n is not None:
+            w = dataclasses.replace(w, n=args.n)
         res = bench_decode(dev, stream, flush, bsa, torch, steps=args.steps, warmup=args.warmup, n=args.n)
     else:
         w = WORKLOADS["bsbr_block_diagonal"]

@@ -7,22 +7,23 @@
 //
 // A query row is a single vector, so the step is a stream over the kept
 // pages' keys and values (HBM/L2 bound, no matrix product to hand to the
-// tensor cores).  The unit of work is a task: 32 consecutive key rows of one
+// tensor cores).  The unit of work is a task: 16 consecutive key rows of one
 // kept page, i.e. one contiguous K run and one contiguous V run of the page's
 // tile for the key/value head.  A thread-block cluster of C CTAs (C = 1..8,
 // chosen on the host from the layout's longest row and the number of query
 // groups, so that short rows spread over many SMs and long batches do not
-// oversubscribe them) serves G query rows of one key/value head (G = 2 when
-// two rows of a group share a route, else 1); the row's tasks are dealt
-// round-robin over the cluster's warps.  Each warp double-buffers its tasks
-// (two bulk copies per task on one mbarrier, the next task's copies issued
-// before the current one is scored), with the page numbers of 32 tasks
-// fetched at once by its lanes.  Scoring: 8 lanes per key row, four rows per
-// step, q held in registers, packed fp32 FMAs; a warp keeps an fp32 online
-// softmax per query (P is not rounded to bf16) and accumulates P V with lanes
-// across d.  The warps' partial (max, sum, o) are merged in shared memory,
-// then the cluster's CTAs' partials are merged by CTA 0 through distributed
-// shared memory; o is stored as bf16 and lse in fp32.
+// exceed the CTAs the GPU holds at once) serves G query rows of one key/value
+// head (G = 2 when two rows of a group share a route, else 1); the row's tasks
+// are dealt round-robin over the cluster's warps.  A warp brings a task's K and
+// V rows into its own buffer with two bulk copies on an mbarrier; small tasks
+// and small buffers keep 24 warps on an SM, which is what hides the copies'
+// latency.  The page numbers of a warp's next 32 tasks are fetched at once by
+// its lanes.  Scoring: 8 lanes per key row, four rows per step, q held in
+// registers, packed fp32 FMAs; a warp keeps an fp32 online softmax per query
+// (P is not rounded to bf16) and accumulates P V with lanes across d.  The
+// warps' partial (max, sum, o) are merged in shared memory, each CTA stores
+// its merged state into CTA 0's (then idle) tile buffers through distributed
+// shared memory, and CTA 0 merges those; o is stored as bf16 and lse in fp32.
 //
 // Positions and page numbers come from device memory: a position outside
 // [0, n) or a page outside [0, num_pages) is not read; the kernel records a
@@ -41,8 +42,8 @@
 namespace bsa {
 namespace dec {
 
-constexpr int kRows = 32;                           // key rows per task
-constexpr int kMaxCluster = 8;                      // portable cluster size
+constexpr int kRows = 16;                           // key rows per task
+constexpr int kMaxCluster = 8;                      // CTAs per cluster at most (portable size)
 constexpr uint64_t kWaitLimitNs = 1000000000ull;    // a copy that takes longer than 1 s is abandoned
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr int kFlagBadIndex = 1, kFlagTimeout = 2;
@@ -64,12 +65,8 @@ struct DecodeParams {
   float scale_log2;
 };
 
-// Warps per CTA: two buffers of a task's K and V tiles per warp, 96 KB of
-// tiles per CTA, so two CTAs fit one SM.
-template <int HD>
-__host__ __device__ constexpr int warps_per_cta() {
-  return HD == 128 ? 3 : 6;
-}
+// Warps per CTA, each with one buffer for its current task's K and V rows.
+constexpr int kWarps = 6;
 template <int HD>
 __host__ __device__ constexpr uint32_t task_tile_bytes() {   // one task's K (or V) rows
   return uint32_t(kRows) * HD * 2;
@@ -128,10 +125,14 @@ __device__ __forceinline__ int cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return int(r);
 }
-// Every thread of every CTA of the cluster: writes before are visible to the
-// cluster's reads after.
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+// Cluster barrier in two halves: every thread of every CTA arrives, then waits
+// for all of them.  With release/acquire, writes before the arrival (shared
+// memory of other CTAs included) are visible after the wait.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Address of the same shared variable in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t peer_addr(const void* p, int rank) {
@@ -139,32 +140,33 @@ __device__ __forceinline__ uint32_t peer_addr(const void* p, int rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
   return a;
 }
-__device__ __forceinline__ float ld_peer_f32(uint32_t a) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-  return v;
+__device__ __forceinline__ void st_peer_f32(uint32_t a, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
-__device__ __forceinline__ int ld_peer_s32(uint32_t a) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
-  return v;
+__device__ __forceinline__ void st_peer_s32(uint32_t a, int v) {
+  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(a), "r"(v) : "memory");
 }
 
 template <int BLK, int HD, int G>
-__global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(const DecodeParams p) {
-  constexpr int W = warps_per_cta<HD>();
+__global__ void __launch_bounds__(kWarps * 32, 4) bsa_decode_kernel(const DecodeParams p) {
+  constexpr int W = kWarps;
   constexpr int PB = BLK / kRows;     // tasks per page
   constexpr int CPL = HD / 8;         // key columns per lane (8 lanes per key row)
   constexpr int DPL = HD / 32;        // o columns per lane
   constexpr uint32_t kTile = task_tile_bytes<HD>();
   constexpr unsigned kAll = 0xffffffffu;
-  extern __shared__ __align__(128) uint8_t dyn[];   // per warp: 2 x (K tile, V tile)
-  __shared__ __align__(8) uint64_t bars[W][2];
+  static_assert(kRows <= 32 && kRows % 4 == 0, "a task's rows map onto a warp's lanes");
+  // Per warp: the K and V rows of its current task.  After the last task the
+  // same buffer holds the warp's partial o (G x HD fp32) and, at CTA 0, two of
+  // the cluster's CTA partial states (o[HD], max, sum per query) behind it.
+  constexpr uint32_t kPartialBytes = G * (HD + 2) * 4;
+  static_assert(G * HD * 4 + 2 * kPartialBytes <= 2 * kTile && (kMaxCluster + 1) / 2 <= W,
+                "a warp's buffer holds its partial o and two CTA partial states");
+  extern __shared__ __align__(128) uint8_t dyn[];
+  __shared__ __align__(8) uint64_t bars[W];
   __shared__ float sp[W][G][kRows];               // scores, then P, of a warp's task
   __shared__ float sm[W][G], sl[W][G];
-  __shared__ float so[W][G][HD];
-  __shared__ float cm[G], cl[G];                  // the CTA's merged partial state
-  __shared__ float co[G][HD];
+  __shared__ int xflags[kMaxCluster];             // at CTA 0: each CTA's flags
   __shared__ int s_flags, s_start, s_len, s_t;
 
   const int C = p.C;
@@ -174,6 +176,11 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
   const int hk = (f0 - b * p.H) / p.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float sl2 = p.scale_log2;
+  // CTA r's partial state for query gq, at CTA 0
+  auto partial = [&](int r, int gq) -> float* {
+    return reinterpret_cast<float*>(dyn + size_t(r >> 1) * 2 * kTile + G * HD * 4 + (r & 1) * kPartialBytes) +
+           gq * (HD + 2);
+  };
   if (threadIdx.x == 0) {
     const int t = p.positions[b];
     int start = 0, len = 0, flags = 0;
@@ -190,8 +197,7 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
     s_flags = flags;
   }
   if (lane == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp][0])) : "memory");
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp][1])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp])) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // this lane's query columns, in registers
@@ -215,8 +221,10 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
   const int T = len * PB;                         // tasks of the row
   const int gw = rank * W + warp, S = C * W;      // this warp's first task, stride
   const int mine = T > gw ? (T - gw + S - 1) / S : 0;
-  uint8_t* wbase = dyn + size_t(warp) * 4 * kTile;
-  const uint32_t bar0 = smem_u32(&bars[warp][0]);
+  uint8_t* wbase = dyn + size_t(warp) * 2 * kTile;
+  const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(wbase);
+  const __nv_bfloat16* vt = kt + kRows * HD;
+  const uint32_t bar = smem_u32(&bars[warp]);
   float m[G], l[G], acc[G][DPL];
 #pragma unroll
   for (int gq = 0; gq < G; ++gq) {
@@ -226,17 +234,13 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
     for (int e = 0; e < DPL; ++e) acc[gq][e] = 0.f;
   }
   // lane x holds the key block and page of local task m0 + x
-  int m0 = -kRows, idx_j = 0, idx_page = -1;
-  // per buffer: first key of the task in it; bit k of `live`: copies in flight into buffer k
-  int u_first0 = 0, u_first1 = 0;
-  uint32_t live = 0;
-  uint32_t phase = 0;                             // bit k: parity of buffer k's next completion
+  int m0 = -32, idx_j = 0, idx_page = -1;
+  uint32_t phase = 0;                             // parity of the buffer's next completion
+  bool live = false;                              // copies in flight into the buffer
   int flags = 0;
 
-  // Issue the copies of local task mt into buffer mt & 1 (nothing for a task
-  // past the token or with a refused page).
-  auto issue = [&](int mt) {
-    if (mt - m0 >= 32) {
+  for (int mt = 0; mt < mine; ++mt) {
+    if (mt - m0 >= 32) {                          // page numbers of the next 32 tasks
       m0 = mt;
       const int x = mt + lane;
       idx_j = 0;
@@ -249,43 +253,27 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
     }
     const int j = __shfl_sync(kAll, idx_j, mt - m0);
     const int page = __shfl_sync(kAll, idx_page, mt - m0);
-    const int part = (gw + mt * S) % PB;
-    const int bi = mt & 1;
-    const int u_first = j * BLK + part * kRows;
-    if (bi) u_first1 = u_first; else u_first0 = u_first;
+    const int u0 = j * BLK + ((gw + mt * S) % PB) * kRows;   // the task's first key
     if (page < 0 || page >= p.num_pages) {
       flags |= kFlagBadIndex;
-      return;
+      continue;
     }
-    if (u_first > t) return;                       // every key of the task is after the token
-    live |= 1u << bi;
-    __syncwarp();                                  // every lane is done with the buffer's last task
-    if (lane == 0) {
-      const uint32_t bar = bar0 + 8u * bi;
-      const size_t off = ((size_t(page) * p.hkv + hk) * BLK + size_t(part) * kRows) * HD;
-      uint8_t* kt = wbase + size_t(bi) * 2 * kTile;
+    if (u0 > t) continue;                         // every key of the task is after the token
+    if (lane == 0) {                              // every lane is done with the last task (warp barrier below)
+      const size_t off = (size_t(page) * p.hkv + hk) * BLK * HD + size_t(u0 - j * BLK) * HD;
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads before the copy
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(2 * kTile) : "memory");
       bulk_load(smem_u32(kt), p.kc + off, kTile, bar);
-      bulk_load(smem_u32(kt + kTile), p.vc + off, kTile, bar);
+      bulk_load(smem_u32(vt), p.vc + off, kTile, bar);
     }
-  };
-
-  if (mine > 0) issue(0);
-  for (int mt = 0; mt < mine; ++mt) {
-    const int bi = mt & 1;
-    if (mt + 1 < mine) issue(mt + 1);
-    if (!((live >> bi) & 1u)) continue;
-    const bool landed = bar_wait(bar0 + 8u * bi, (phase >> bi) & 1u);
-    phase ^= 1u << bi;
-    live &= ~(1u << bi);
-    if (!__all_sync(kAll, landed)) {
+    live = true;
+    const bool landed = bar_wait(bar, phase);
+    if (!__all_sync(kAll, landed)) {              // the drain below waits on the same phase
       flags |= kFlagTimeout;
       break;
     }
-    const __nv_bfloat16* kt = reinterpret_cast<const __nv_bfloat16*>(wbase + size_t(bi) * 2 * kTile);
-    const __nv_bfloat16* vt = kt + kRows * HD;
-    const int u0 = bi ? u_first1 : u_first0;       // the task's first key
+    phase ^= 1u;
+    live = false;
     // ---- scores: rows 4 * step + sub, columns pc * CPL ..
 #pragma unroll 2
     for (int step = 0; step < kRows / 4; ++step) {
@@ -317,17 +305,17 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
       }
     }
     __syncwarp();
-    // ---- online softmax per query; lane x owns key row x of the task
+    // ---- online softmax per query; lane x < kRows owns key row x of the task
 #pragma unroll
     for (int gq = 0; gq < G; ++gq) {
-      const float s = sp[warp][gq][lane];
+      const float s = lane < kRows ? sp[warp][gq][lane] : -INFINITY;
       float bm = s;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(kAll, bm, off));
       const float m_new = fmaxf(m[gq], bm);        // finite: the task's first key is allowed
       const float alpha = ex2(m[gq] - m_new);      // 0 while m is -inf
-      const float pv = ex2(s - m_new);             // 0 for a disallowed key
-      sp[warp][gq][lane] = pv;
+      const float pv = ex2(s - m_new);             // 0 for a disallowed key or an idle lane
+      if (lane < kRows) sp[warp][gq][lane] = pv;
       float psum = pv;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(kAll, psum, off);
@@ -359,14 +347,12 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
     __syncwarp();
   }
   // leave no copy in flight into shared memory
-  if (lane == 0) {
-#pragma unroll
-    for (int bi = 0; bi < 2; ++bi)
-      if (((live >> bi) & 1u) && !bar_wait(bar0 + 8u * bi, (phase >> bi) & 1u)) flags |= kFlagTimeout;
-  }
+  if (lane == 0 && live && !bar_wait(bar, phase)) flags |= kFlagTimeout;
+  __syncwarp();
   flags = __reduce_or_sync(kAll, flags);
   if (lane == 0 && flags) atomicOr(&s_flags, flags);
-  // ---- merge the warps' partial softmax states
+  // ---- merge the warps' partial softmax states (o over the warp's own buffer)
+  float* so = reinterpret_cast<float*>(wbase);
 #pragma unroll
   for (int gq = 0; gq < G; ++gq) {
     if (lane == 0) {
@@ -374,9 +360,13 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
       sl[warp][gq] = l[gq];
     }
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) so[warp][gq][lane * DPL + e] = acc[gq][e];
+    for (int e = 0; e < DPL; ++e) so[gq * HD + lane * DPL + e] = acc[gq][e];
   }
   __syncthreads();
+  // Every CTA of the cluster is done with its tiles (CTA 0's buffers take the
+  // partial states next).
+  cluster_arrive();
+  cluster_wait();
   for (int c = threadIdx.x; c < G * HD; c += W * 32) {
     const int gq = c / HD, col = c % HD;
     float M = -INFINITY;
@@ -387,38 +377,40 @@ __global__ void __launch_bounds__(warps_per_cta<HD>() * 32) bsa_decode_kernel(co
     for (int w = 0; w < W; ++w) {
       const float wt = (M == -INFINITY) ? 0.f : ex2(sm[w][gq] - M);
       Lsum += wt * sl[w][gq];
-      v += wt * so[w][gq][col];
+      v += wt * reinterpret_cast<const float*>(dyn + size_t(w) * 2 * kTile)[gq * HD + col];
     }
-    co[gq][col] = v;
+    // this CTA's partial state into CTA 0's shared memory
+    float* dst = partial(rank, gq);
+    st_peer_f32(peer_addr(dst + col, 0), v);
     if (col == 0) {
-      cm[gq] = M;
-      cl[gq] = Lsum;
+      st_peer_f32(peer_addr(dst + HD, 0), M);
+      st_peer_f32(peer_addr(dst + HD + 1, 0), Lsum);
     }
   }
-  // ---- merge the cluster's CTAs (CTA 0 reads the others' shared memory)
-  cluster_sync();
-  if (rank == 0) {
-    int all_flags = 0;
-    for (int r = 0; r < C; ++r) all_flags |= ld_peer_s32(peer_addr(&s_flags, r));
-    for (int c = threadIdx.x; c < G * HD; c += W * 32) {
-      const int gq = c / HD, col = c % HD;
-      float M = -INFINITY;
-      for (int r = 0; r < C; ++r) M = fmaxf(M, ld_peer_f32(peer_addr(&cm[gq], r)));
-      float Lsum = 0.f, v = 0.f;
-      for (int r = 0; r < C; ++r) {
-        const float wt = (M == -INFINITY) ? 0.f : ex2(ld_peer_f32(peer_addr(&cm[gq], r)) - M);
-        Lsum += wt * ld_peer_f32(peer_addr(&cl[gq], r));
-        v += wt * ld_peer_f32(peer_addr(&co[gq][col], r));
-      }
-      const bool ok = Lsum > 0.f && all_flags == 0;
-      p.o[size_t(f0 + gq) * HD + col] = __float2bfloat16_rn(ok ? v / Lsum : 0.f);
-      if (col == 0) p.lse[f0 + gq] = ok ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+  if (threadIdx.x == 0) st_peer_s32(peer_addr(&xflags[rank], 0), s_flags);
+  cluster_arrive();
+  cluster_wait();                                 // the partial states have landed at CTA 0
+  if (rank != 0) return;
+  int all_flags = 0;
+  for (int r = 0; r < C; ++r) all_flags |= xflags[r];
+  for (int c = threadIdx.x; c < G * HD; c += W * 32) {
+    const int gq = c / HD, col = c % HD;
+    float M = -INFINITY;
+    for (int r = 0; r < C; ++r) M = fmaxf(M, partial(r, gq)[HD]);
+    float Lsum = 0.f, v = 0.f;
+    for (int r = 0; r < C; ++r) {
+      const float* x = partial(r, gq);
+      const float wt = (M == -INFINITY) ? 0.f : ex2(x[HD] - M);
+      Lsum += wt * x[HD + 1];
+      v += wt * x[col];
     }
-    if (threadIdx.x == 0 && all_flags)
-      atomicOr(p.status, (all_flags & kFlagTimeout ? kStatusTimeout : 0u) |
-                             (all_flags & kFlagBadIndex ? kStatusBadIndex : 0u));
+    const bool ok = Lsum > 0.f && all_flags == 0;
+    p.o[size_t(f0 + gq) * HD + col] = __float2bfloat16_rn(ok ? v / Lsum : 0.f);
+    if (col == 0) p.lse[f0 + gq] = ok ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
   }
-  cluster_sync();                                   // CTA 0 is done reading the others
+  if (threadIdx.x == 0 && all_flags)
+    atomicOr(p.status, (all_flags & kFlagTimeout ? kStatusTimeout : 0u) |
+                           (all_flags & kFlagBadIndex ? kStatusBadIndex : 0u));
 }
 
 // CTAs per cluster: enough warps for one task each on the longest row, cut
@@ -433,29 +425,32 @@ inline int cluster_size(int groups, int max_row, int tasks_per_page, int warps, 
 template <int BLK, int HD, int G>
 int launch_g(DecodeParams p, int heads, int max_row, cudaStream_t s) {
   auto kern = bsa_decode_kernel<BLK, HD, G>;
-  constexpr int W = warps_per_cta<HD>();
-  const int smem = W * 4 * int(task_tile_bytes<HD>());
+  constexpr int W = kWarps;
+  const int smem = W * 2 * int(task_tile_bytes<HD>());
   // the attribute is a property of the function: set it once per device
   static std::mutex mu;
   static bool done[64] = {};
-  static int sms[64] = {};
+  static int resident[64] = {};                   // CTAs the GPU holds at once
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= 64) return set_error(BSA_ERR_CUDA, "cannot query the device");
-  int n_sm = 0;
+  int n_resident = 0;
   {
     std::lock_guard<std::mutex> lock(mu);
     if (!done[dev]) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode smem: ") + cudaGetErrorString(e));
-      e = cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
-      if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode SMs: ") + cudaGetErrorString(e));
+      int n_sm = 0, per_sm = 0;
+      e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+      if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, W * 32, smem);
+      if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("decode occupancy: ") + cudaGetErrorString(e));
+      resident[dev] = std::max(1, n_sm * per_sm);
       done[dev] = true;
     }
-    n_sm = sms[dev];
+    n_resident = resident[dev];
   }
   const int groups = heads / G;
-  p.C = cluster_size(groups, max_row, BLK / kRows, W, 2 * n_sm);
+  p.C = cluster_size(groups, max_row, BLK / kRows, W, n_resident);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(groups * p.C), 1, 1);
   cfg.blockDim = dim3(W * 32, 1, 1);
