@@ -407,6 +407,21 @@ def main():
     ms_per_step = total_ms / args.steps
     value = sharding.aggregate_rate(flops * args.steps, world, total_ms * 1e-3) / 1e12
     clocks = sampler.summary(wall0 - 0.05, wall1 + 0.05)
+    # distribution of the cold (flushed) steps above, and a warm figure taken
+    # after the timed region: back-to-back launches with no flush between them
+    cold = sorted(step_ms)
+    warm_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(20)]
+    for a_ev, b_ev in warm_ev:
+        a_ev.record(stream)
+        fwd()
+        b_ev.record(stream)
+    torch.cuda.synchronize()
+    warm = sorted(a_ev.elapsed_time(b_ev) for a_ev, b_ev in warm_ev)
+    step_stats = {"cold_median": cold[len(cold) // 2], "cold_p10": cold[len(cold) // 10],
+                  "cold_p90": cold[min(len(cold) - 1, (9 * len(cold)) // 10)],
+                  "warm_median": warm[len(warm) // 2],
+                  "note": "per-launch ms on this rank; cold = 256 MiB written before each timed launch, "
+                          "warm = 20 launches back to back after the timed region"}
 
     if args.only_device:
         if rank == 0:
@@ -504,7 +519,7 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "step_ms": step_stats, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic N(0,1) bf16 from numpy default_rng, q/k/v seeds 3r/3r+1/3r+2 on rank r; "
                     "layout seed 17",
