@@ -209,8 +209,10 @@ int bsa_forward_noalloc(const void* q, const void* k, const void* v,
  * 4-byte aligned; num_pages must be the number of pages the caches hold.  A
  * position outside [0, n) or a page outside [0, num_pages) read on the device
  * is not dereferenced: the rows it concerns get o = 0, lse = -inf and
- * bsa_get_status then reports BSA_ERR_SHAPE.  Launches one kernel and returns
- * after enqueueing it; no allocation, no synchronisation. */
+ * bsa_get_status then reports BSA_ERR_SHAPE.  Launches one kernel (a
+ * thread-block cluster launch: the CTAs of a cluster split a row's kept pages
+ * and merge their partial softmax states on chip) and returns after
+ * enqueueing it; no allocation, no workspace, no synchronisation. */
 int bsa_decode(const void* q, const void* k_cache, const void* v_cache,
                const int32_t* page_table, int max_blocks, int num_pages,
                const int32_t* positions, const bsa_layout* layout, int batch,
