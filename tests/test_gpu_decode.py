@@ -86,6 +86,25 @@ def test_decode_full_32k_dyadic():
     lay.close()
 
 
+def test_decode_cluster_shapes():
+    """The launch shapes the host picks at the ends of its range: a one-block
+    route (BSBR's block-diagonal layout: four tasks a row, one CTA per
+    cluster) and so many query groups (25 sequences x 8 key/value heads) that
+    the clusters shrink to fit the GPU at once (to two CTAs on a 148-SM
+    B200, the shape of a batch-32 decode of the 32K route)."""
+    for kind, n, B, batch, H, hkv, d, pat in (
+            (OL.BAND_GLOBAL, 1024, 64, 2, 4, 2, 64, dict(window=0, global_first=0)),
+            (OL.DYADIC, 2048, 64, 25, 16, 8, 128, dict(window=2, global_first=1, dyadic_kmin=2))):
+        scale = 1.0 / math.sqrt(d)
+        lay, sets, dev_t, host = _setup(kind, n, B, 1, batch, H, hkv, d, pat, seed=11)
+        rng = np.random.default_rng(12)
+        for positions in ([n - 1] * batch, [int(x) for x in rng.integers(0, n, batch)]):
+            o, lse, o_ref, lse_ref = _step(lay, sets, dev_t, host, batch, H, d, B, positions, scale)
+            assert_close(o, lse, o_ref, lse_ref, f"{kind} n{n} batch {batch}")
+        bsa.bsa_get_status(lay.handle)
+        lay.close()
+
+
 def test_decode_long_rows_many_tasks_per_warp():
     """Full causal rows of up to 512 pages: each warp of a cluster takes more
     than 32 tasks of 32 key rows, so its page numbers are fetched in several
