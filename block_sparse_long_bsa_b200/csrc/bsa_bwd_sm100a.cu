@@ -73,6 +73,7 @@ struct Params {
   float* dk;
   float* dv;
   uint32_t* status;
+  uint32_t* work_counter;   // next unclaimed item of the launched kernel (zeroed before its launch)
   int n, nb, L, heads, kv_heads, group, pack, n_steps;   // n_steps = group / pack head steps per key/value head
   int items;         // work items of the launched kernel
   float scale, scale_log2;
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(256) bsa_bwd_clear_kernel(const Params p, int 
 
 // ---------------------------------------------------------------- dQ
 // Persistent: one CTA per SM walks query tiles (head group by head group,
-// longest row first inside one, every gridDim-th).  Warp 0 decodes each tile
+// longest row first inside one; CTAs claim them in order through a counter).  Warp 0 decodes each tile
 // into a ring of shared-memory slots (read by the other warps) and loads its
 // Q, dO, K and V tiles.  A tile's kept blocks are taken 128 keys at a time
 // (two 64-key chunks: two blocks for B = 64, one for B = 128; a lone last
@@ -349,9 +350,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(dst + a * S::kAtomKV + h * kChunk * 128, m, b, a * 64, key0, it.kvh);
         }
       };
-      for (int k = 0, x = blockIdx.x; ok; ++k, x += gridDim.x) {
+      // items are claimed in list order through the counter, so every CTA
+      // ends within about one item of the others
+      int x = int(atomicAdd(p.work_counter, 1u));
+      for (int k = 0; ok; ++k) {
         if (k >= kRing && !(ok = ctl.wait(bar(S::kBItemFree + k % kRing), uint32_t((k - kRing) / kRing) & 1u))) break;
         const DqSlot it = dq_decode<BLK>(p, x);
+        // the next claim's latency overlaps this item's hand-over and loads
+        const int x_next = it.last ? x : int(atomicAdd(p.work_counter, 1u));
         volatile int* v = reinterpret_cast<volatile int*>(ring + (k % kRing) * 32);
         v[0] = it.i;
         v[1] = it.h0;
@@ -362,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         v[6] = it.last;
         mbar_arrive(bar(S::kBItem + k % kRing));
         if (it.last) break;
+        x = x_next;
         if (it.nch == 0) continue;
         const int b = xi & 1;
         if (xi >= 2 && !(ok = ctl.wait(bar(S::kBQFree + b), uint32_t((xi - 2) >> 1) & 1u))) break;
@@ -620,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- dK, dV
 // Persistent: one CTA per SM walks work items (key/value head, column
 // segment, query-head step, 64-key chunk of a key block; head by head,
-// longest segments first inside one, every gridDim-th).  A segment lists up to 16 query blocks whose rows keep
+// longest segments first inside one; CTAs claim them in order through a counter).  A segment lists up to 16 query blocks whose rows keep
 // the key block (the transposed layout).  Warp 0 decodes each item into a
 // ring of shared-memory slots and loads its tiles.  Per query tile t:
 // S = Q K^T and dP = dO V^T (M = 128 query rows) into TMEM buffer t & 1; the
@@ -758,11 +765,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int t = 0, y = 0;
       int k = 0;
-      for (int x = blockIdx.x; ok; x += gridDim.x) {
+      // items are claimed in list order through the counter, so every CTA
+      // ends within about one item of the others
+      int x = int(atomicAdd(p.work_counter, 1u));
+      while (ok) {
         DkvSlot it{};
         int e0 = 0;
         const bool end = x >= p.items;
-        if (!end && !dkv_decode<BLK>(p, x, it, e0)) continue;
+        if (!end && !dkv_decode<BLK>(p, x, it, e0)) {
+          x = int(atomicAdd(p.work_counter, 1u));
+          continue;
+        }
+        // the next claim's latency overlaps this item's hand-over and loads
+        const int x_next = end ? x : int(atomicAdd(p.work_counter, 1u));
         if (k >= kRing && !(ok = ctl.wait(bar(S::kBItemFree + k % kRing), uint32_t((k - kRing) / kRing) & 1u))) break;
         volatile int* v = reinterpret_cast<volatile int*>(ring + (k % kRing) * S::kSlotBytes);
         v[0] = it.kvh;
@@ -789,6 +804,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++t;
         }
         ++k;
+        x = x_next;
       }
       if (!ok) {
         for (int e = (t > 2 ? t - 2 : 0); e < t; ++e) wait_drain(bar(S::kBQ + (e & 1)), uint32_t(e >> 1) & 1u, kDrainNs);
@@ -1047,9 +1063,17 @@ int launch_instance(const Launch& a, const bwd::Params& p) {
   bwd::Params pq = p, pk = p;
   pq.items = a.items_dq;
   pk.items = a.items_dkv;
-  if (a.items_dq > 0) kq<<<a.items_dq < a.sms ? a.items_dq : a.sms, bwd::kThreads, smem_q, a.stream>>>(mq, mdo, mk2, mv2, pq);
-  if (a.items_dkv > 0)
+  // the two product kernels share one item counter, cleared before each
+  if (a.items_dq > 0) {
+    e = cudaMemsetAsync(pq.work_counter, 0, sizeof(uint32_t), a.stream);
+    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing the item counter: ") + cudaGetErrorString(e));
+    kq<<<a.items_dq < a.sms ? a.items_dq : a.sms, bwd::kThreads, smem_q, a.stream>>>(mq, mdo, mk2, mv2, pq);
+  }
+  if (a.items_dkv > 0) {
+    e = cudaMemsetAsync(pk.work_counter, 0, sizeof(uint32_t), a.stream);
+    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing the item counter: ") + cudaGetErrorString(e));
     kkv<<<a.items_dkv < a.sms ? a.items_dkv : a.sms, bwd::kThreads, smem_kv, a.stream>>>(mq, mdo, mk, mv, pk);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
   return BSA_OK;
@@ -1107,6 +1131,11 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   p.dk = dk;
   p.dv = dv;
   p.status = layout->d_status;
+  {
+    // one of the layout's work counters, taken in turn with its forwards
+    const uint32_t call = const_cast<bsa_layout*>(layout)->calls.fetch_add(1, std::memory_order_relaxed);
+    p.work_counter = layout->d_status + 64 + size_t(call % kWorkCounters) * 32;
+  }
   p.n = n;
   p.nb = layout->nb;
   p.L = layout->L;

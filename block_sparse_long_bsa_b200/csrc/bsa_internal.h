@@ -33,7 +33,7 @@ struct bsa_layout {
   const int32_t* d_seg_ptr = nullptr;
   const int32_t* d_segs = nullptr;
   uint32_t* d_status = nullptr;   // bit 0: a device wait ran out
-  std::atomic<uint32_t> calls{0};  // forwards launched (picks each call's work counter)
+  std::atomic<uint32_t> calls{0};  // forwards and backwards launched (picks each call's work counter)
 };
 
 namespace bsa {
@@ -53,8 +53,9 @@ constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusBadIndex = 2u;   // a decode position or page number was out of range
 // The status block that follows a layout's arrays holds the status word at
 // word 0 and, from byte 256 on, kWorkCounters work counters, one per 128-byte
-// line: forward number c of a layout uses counter c % kWorkCounters, so up to
-// that many forwards on one layout may be in flight at once.  The
+// line: call number c of a layout (forward or backward) uses counter
+// c % kWorkCounters, so up to that many calls on one layout may be in flight
+// at once.  The
 // allocation-free scratch has one counter, at word 32.
 constexpr int kWorkCounters = 64;
 constexpr size_t kStatusBlockBytes = 256 + size_t(kWorkCounters) * 128;

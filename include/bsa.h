@@ -140,8 +140,8 @@ int bsa_layout_csc(const bsa_layout* layout, const int32_t** col_ptr,
  * o and lse must not overlap the inputs.  Enqueues a 4-byte clear of a work
  * counter and one kernel; returns after enqueueing them.  Each call takes the
  * next of 64 work counters held in the layout's device block, so forwards
- * with the same layout may run at the same time on different streams (up to
- * 64 in flight at once).  A device-side wait that runs out (never expected)
+ * (and backwards) with the same layout may run at the same time on different
+ * streams (up to 64 in flight at once).  A device-side wait that runs out (never expected)
  * makes the kernel return early and is reported by bsa_get_status. */
 int bsa_forward(const void* q, const void* k, const void* v,
                 const bsa_layout* layout, int B, int n, int heads, int kv_heads,
@@ -233,11 +233,15 @@ int bsa_decode(const void* q, const void* k_cache, const void* v_cache,
  * dv [kv_heads][n][d] fp32; workspace [heads][n] fp32 (receives D).  All
  * device memory, caller-owned, not overlapping.  Requirements as for
  * bsa_forward (checked before launch; errors launch nothing), plus dout, dq,
- * dk, dv 16-byte aligned and workspace 4-byte aligned.  Enqueues two clears
- * (dk, dv) and three kernels (D, dq, dk/dv) on the stream and returns; the
- * dk/dv kernel adds its partial sums in fp32, so their summation order (and
- * last bits) may differ from run to run.  A wait that runs out is reported
- * by bsa_get_status as for the forward. */
+ * dk, dv 16-byte aligned and workspace 4-byte aligned.  Enqueues the clear
+ * of dk and dv (two memsets, or a kernel clearing only the rows that several
+ * CTAs add into), a 4-byte clear of a work counter before each of the dq and
+ * dk/dv kernels, and three kernels (D, dq, dk/dv) on the stream, and returns.
+ * The work counter is the next of the layout's 64, taken in turn with its
+ * forwards, so up to 64 forwards and backwards on one layout may be in
+ * flight at once.  The dk/dv kernel adds its partial sums in fp32, so their
+ * summation order (and last bits) may differ from run to run.  A wait that
+ * runs out is reported by bsa_get_status as for the forward. */
 int bsa_backward(const void* q, const void* k, const void* v, const void* o,
                  const float* lse, const void* dout, const bsa_layout* layout,
                  int B, int n, int heads, int kv_heads, int d, float scale,
