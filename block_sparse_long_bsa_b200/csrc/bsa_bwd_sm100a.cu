@@ -148,27 +148,51 @@ struct Idle {
 };
 
 // ---------------------------------------------------------------- D = rowsum(dO * o)
-// One warp per query row: D_t = sum_u P_tu dP_tu, which equals <dO_t, o_t>.
+// D_t = sum_u P_tu dP_tu, which equals <dO_t, o_t>.  A row is read with
+// 16-byte loads by HD / 8 lanes; a warp takes kRowdotPasses groups of rows and
+// issues all of their loads before any arithmetic, so each thread keeps
+// several loads in flight (the pass is bound by HBM).
+constexpr int kRowdotPasses = 4;
+template <int HD>
+__host__ __device__ constexpr int rowdot_rows_per_cta() {
+  return 8 * (32 / (HD / 8)) * kRowdotPasses;   // 8 warps x rows per pass x passes
+}
 template <int HD>
 __global__ void __launch_bounds__(256) bsa_bwd_rowdot_kernel(const __nv_bfloat16* o, const __nv_bfloat16* dout,
                                                              float* dsum, size_t rows) {
-  const size_t row = size_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  float acc = 0.f;
+  constexpr int kLanesPerRow = HD / 8;
+  constexpr int kRowsPerPass = 32 / kLanesPerRow;
+  const int lane = threadIdx.x & 31, sub = lane / kLanesPerRow, part = lane % kLanesPerRow;
+  const size_t row0 = size_t(blockIdx.x) * rowdot_rows_per_cta<HD>() +
+                      size_t(threadIdx.x >> 5) * (kRowsPerPass * kRowdotPasses);
+  uint4 a[kRowdotPasses], b[kRowdotPasses];
 #pragma unroll
-  for (int c = lane * 4; c < HD; c += 128) {
-    const uint2 a = *reinterpret_cast<const uint2*>(o + row * HD + c);
-    const uint2 b = *reinterpret_cast<const uint2*>(dout + row * HD + c);
-    const float2 a0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.x));
-    const float2 a1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&a.y));
-    const float2 b0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.x));
-    const float2 b1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&b.y));
-    acc = fmaf(a0.x, b0.x, fmaf(a0.y, b0.y, fmaf(a1.x, b1.x, fmaf(a1.y, b1.y, acc))));
+  for (int ps = 0; ps < kRowdotPasses; ++ps) {
+    const size_t row = row0 + size_t(ps) * kRowsPerPass + sub;
+    if (row < rows) {
+      a[ps] = *reinterpret_cast<const uint4*>(o + row * HD + part * 8);
+      b[ps] = *reinterpret_cast<const uint4*>(dout + row * HD + part * 8);
+    } else {
+      a[ps] = make_uint4(0u, 0u, 0u, 0u);
+      b[ps] = make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) dsum[row] = acc;
+  for (int ps = 0; ps < kRowdotPasses; ++ps) {
+    const uint32_t wa[4] = {a[ps].x, a[ps].y, a[ps].z, a[ps].w};
+    const uint32_t wb[4] = {b[ps].x, b[ps].y, b[ps].z, b[ps].w};
+    float acc = 0.f;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[h]));
+      const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[h]));
+      acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+    }
+#pragma unroll
+    for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    const size_t row = row0 + size_t(ps) * kRowsPerPass + sub;
+    if (part == 0 && row < rows) dsum[row] = acc;
+  }
 }
 
 // ---------------------------------------------------------------- dk, dv clear
@@ -1057,7 +1081,7 @@ int launch_instance(const Launch& a, const bwd::Params& p) {
     if (e == cudaSuccess) e = cudaMemsetAsync(p.dv, 0, grad_kv, a.stream);
     if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing dk, dv: ") + cudaGetErrorString(e));
   }
-  const unsigned rows_grid = unsigned((a.dq_rows + 7) / 8);
+  const unsigned rows_grid = unsigned((a.dq_rows + bwd::rowdot_rows_per_cta<HD>() - 1) / bwd::rowdot_rows_per_cta<HD>());
   bwd::bsa_bwd_rowdot_kernel<HD><<<rows_grid, 256, 0, a.stream>>>(
       static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.dsum, a.dq_rows);
   bwd::Params pq = p, pk = p;
