@@ -35,7 +35,8 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "B
                 7: "BSA_ERR_DEVICE_TIMEOUT"}
 
 EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_csc", "bsa_layout_order",
-            "bsa_layout_segments", "bsa_forward", "bsa_forward_noalloc", "bsa_backward", "bsa_decode",
+            "bsa_layout_segments", "bsa_forward", "bsa_forward_host", "bsa_forward_noalloc", "bsa_backward",
+            "bsa_decode",
             "bsa_bsbr_workspace_bytes", "bsa_bsbr_retrieval", "bsa_get_status", "bsa_debug_timeout_probe",
             "bsa_free", "bsa_last_error"]
 
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH):
         lib.bsa_forward.restype = I
         lib.bsa_forward_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P]
         lib.bsa_forward_noalloc.restype = I
+        lib.bsa_forward_host.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P, P, P, P, P, I, P]
+        lib.bsa_forward_host.restype = I
         lib.bsa_decode.argtypes = [P, P, P, P, I, I, P, P, I, I, I, I, F, P, P, P]
         lib.bsa_decode.restype = I
         lib.bsa_backward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, P, P, P]
@@ -213,6 +216,17 @@ def bsa_forward(q, k, v, layout: int, B: int, n: int, heads: int, kv_heads: int,
     lib = load_library()
     _check(lib.bsa_forward(_ptr(q), _ptr(k), _ptr(v), layout, B, n, heads, kv_heads, d,
                            ctypes.c_float(scale), _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def bsa_forward_host(q_host, k_host, v_host, layout: int, B: int, n: int, heads: int, kv_heads: int, d: int,
+                     scale: float, q, k, v, o, lse, o_host, lse_host, groups: int = 8, stream=None) -> None:
+    """Forward from and to host memory (see include/bsa.h): copies in head
+    groups overlap the other groups' compute; synchronise ``stream`` before
+    reading ``o_host`` and ``lse_host``."""
+    lib = load_library()
+    _check(lib.bsa_forward_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), layout, B, n, heads, kv_heads, d,
+                                ctypes.c_float(scale), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                _ptr(o_host), _ptr(lse_host), groups, _stream(stream)))
 
 
 def bsa_forward_noalloc(q, k, v, layout: int, B: int, n: int, heads: int, kv_heads: int, d: int,

@@ -5,8 +5,10 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "bsa_internal.h"
 
@@ -189,9 +191,8 @@ int bsa_layout_segments(const bsa_layout* layout, const int32_t** seg_ptr, const
   return BSA_OK;
 }
 
-int bsa_forward(const void* q, const void* k, const void* v, const bsa_layout* layout, int B,
-                int n, int heads, int kv_heads, int d, float scale, void* o, float* lse,
-                void* stream) {
+static int check_forward(const void* q, const void* k, const void* v, const bsa_layout* layout, int B, int n,
+                         int heads, int kv_heads, int d, float scale, const void* o, const float* lse) {
   int st = check_device(layout);
   if (st != BSA_OK) return st;
   if (B != layout->B || n != layout->n)
@@ -209,8 +210,113 @@ int bsa_forward(const void* q, const void* k, const void* v, const bsa_layout* l
   if (!aligned(lse, 4)) return set_error(BSA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (int64_t(heads) * (int64_t(n + B - 1) / B) > INT32_MAX)
     return set_error(BSA_ERR_SHAPE, "too many (head, block) work items");
+  return BSA_OK;
+}
+
+int bsa_forward(const void* q, const void* k, const void* v, const bsa_layout* layout, int B,
+                int n, int heads, int kv_heads, int d, float scale, void* o, float* lse,
+                void* stream) {
+  const int st = check_forward(q, k, v, layout, B, n, heads, kv_heads, d, scale, o, lse);
+  if (st != BSA_OK) return st;
   bsa::ForwardArgs a{q, k, v, o, lse, layout, B, n, heads, kv_heads, d, scale, stream, 0, 0};
   return bsa::launch_forward(a);
+}
+
+// Two copy streams per device (host to device, device to host), created on
+// first use and kept for the process; every call orders its copies against
+// the caller's stream with events, so calls may share them.
+static int copy_streams(int dev, cudaStream_t* up, cudaStream_t* down) {
+  static std::mutex mu;
+  static cudaStream_t streams[64][2] = {};
+  if (dev < 0 || dev >= 64) return set_error(BSA_ERR_CUDA, "device index out of range");
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < 2; ++i) {
+    if (!streams[dev][i]) {
+      const cudaError_t e = cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking);
+      if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("copy stream: ") + cudaGetErrorString(e));
+    }
+  }
+  *up = streams[dev][0];
+  *down = streams[dev][1];
+  return BSA_OK;
+}
+
+int bsa_forward_host(const void* q_host, const void* k_host, const void* v_host, const bsa_layout* layout,
+                     int B, int n, int heads, int kv_heads, int d, float scale, void* q, void* k, void* v,
+                     void* o, float* lse, void* o_host, float* lse_host, int groups, void* stream) {
+  int st = check_forward(q, k, v, layout, B, n, heads, kv_heads, d, scale, o, lse);
+  if (st != BSA_OK) return st;
+  if (!q_host || !k_host || !v_host || !o_host || !lse_host)
+    return set_error(BSA_ERR_INVALID_ARG, "null host pointer");
+  if (groups < 1) return set_error(BSA_ERR_INVALID_ARG, "groups must be >= 1");
+  // Groups are runs of whole key/value heads whose first query head maps to
+  // layout head 0, so each group is a forward of its own: `unit` key/value
+  // heads is the smallest such step.
+  const int g = heads / kv_heads;
+  int a0 = g, b0 = layout->L;
+  while (b0) {
+    const int t = a0 % b0;
+    a0 = b0;
+    b0 = t;
+  }
+  const int unit = layout->L / a0;
+  const int units = kv_heads / unit;
+  const int G = groups < units ? groups : units;
+  cudaStream_t up = nullptr, down = nullptr;
+  st = copy_streams(layout->device, &up, &down);
+  if (st != BSA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t q_head = size_t(n) * d * 2, kv_head = q_head, lse_head = size_t(n) * sizeof(float);
+  std::vector<cudaEvent_t> ev(2 * size_t(G) + 2, nullptr);
+  cudaError_t e = cudaSuccess;
+  for (auto& x : ev)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming);
+  auto fail = [&](const char* what) {
+    for (auto x : ev)
+      if (x) cudaEventDestroy(x);
+    return set_error(BSA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  };
+  if (e != cudaSuccess) return fail("events");
+  // the copies start after the caller's earlier work on its stream
+  e = cudaEventRecord(ev[0], s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(up, ev[0], 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(down, ev[0], 0);
+  if (e != cudaSuccess) return fail("ordering the copies");
+  auto at = [](const void* p, size_t off) { return static_cast<const char*>(p) + off; };
+  auto at_mut = [](void* p, size_t off) { return static_cast<char*>(p) + off; };
+  for (int i = 0; i < G; ++i) {
+    const int u0 = int(int64_t(units) * i / G), u1 = int(int64_t(units) * (i + 1) / G);
+    const int kv0 = u0 * unit, kvn = (u1 - u0) * unit, h0 = kv0 * g, hn = kvn * g;
+    const size_t qo = size_t(h0) * q_head, qb = size_t(hn) * q_head;
+    const size_t ko = size_t(kv0) * kv_head, kb = size_t(kvn) * kv_head;
+    e = cudaMemcpyAsync(at_mut(q, qo), at(q_host, qo), qb, cudaMemcpyHostToDevice, up);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(at_mut(k, ko), at(k_host, ko), kb, cudaMemcpyHostToDevice, up);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(at_mut(v, ko), at(v_host, ko), kb, cudaMemcpyHostToDevice, up);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[1 + 2 * i], up);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev[1 + 2 * i], 0);
+    if (e != cudaSuccess) return fail("host-to-device copy");
+    bsa::ForwardArgs a{at(q, qo), at(k, ko), at(v, ko), at_mut(o, qo),
+                       reinterpret_cast<float*>(at_mut(lse, size_t(h0) * lse_head)), layout, B, n, hn, kvn, d,
+                       scale, stream, 0, 0};
+    st = bsa::launch_forward(a);
+    if (st != BSA_OK) {
+      for (auto x : ev) cudaEventDestroy(x);
+      return st;
+    }
+    e = cudaEventRecord(ev[2 + 2 * i], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(down, ev[2 + 2 * i], 0);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(at_mut(o_host, qo), at(o, qo), qb, cudaMemcpyDeviceToHost, down);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(at_mut(lse_host, size_t(h0) * lse_head), at(lse, size_t(h0) * lse_head),
+                          size_t(hn) * lse_head, cudaMemcpyDeviceToHost, down);
+    if (e != cudaSuccess) return fail("device-to-host copy");
+  }
+  // the caller's stream completes after the last copy back
+  e = cudaEventRecord(ev[2 * size_t(G) + 1], down);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, ev[2 * size_t(G) + 1], 0);
+  if (e != cudaSuccess) return fail("ordering the copies back");
+  for (auto x : ev) cudaEventDestroy(x);   // released once their work completes
+  return BSA_OK;
 }
 
 int bsa_debug_timeout_probe(const bsa_layout* layout, int d, uint64_t timeout_ns, void* stream) {

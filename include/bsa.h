@@ -160,6 +160,26 @@ int bsa_get_status(const bsa_layout* layout, void* stream);
 int bsa_debug_timeout_probe(const bsa_layout* layout, int d, uint64_t timeout_ns,
                             void* stream);
 
+/* The forward from and to host memory (the end-to-end form of bsa_forward):
+ * q, k, v are copied from q_host, k_host, v_host into the caller's device
+ * buffers q, k, v, the forward runs, and o, lse are copied back into o_host,
+ * lse_host.  The work is cut into `groups` runs of whole key/value heads (at
+ * most kv_heads; fewer when layout heads require coarser runs, since every
+ * run must start at a query head of layout head 0), and run i + 1's
+ * host-to-device copies, run i's forward and run i - 1's device-to-host
+ * copies proceed at the same time: two copy streams of the library (created
+ * once per device, ordered against `stream` with events) carry the copies,
+ * `stream` the forwards.  Everything is enqueued after the work already on
+ * `stream`, and `stream` completes only after the last copy back, so
+ * synchronising `stream` makes o_host and lse_host valid.  Layouts and
+ * requirements as for bsa_forward, plus host pointers non-null (page-locked
+ * host memory lets the copies overlap; pageable memory works but serialises
+ * them) and groups >= 1.  No device allocation. */
+int bsa_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                     const bsa_layout* layout, int B, int n, int heads, int kv_heads,
+                     int d, float scale, void* q, void* k, void* v, void* o, float* lse,
+                     void* o_host, float* lse_host, int groups, void* stream);
+
 /* Forward pass for callers that cannot allocate device memory.  This call has
  * no counterpart on the pages that define the method; it exists for processes
  * whose device memory belongs to someone else (a serving framework that
