@@ -189,3 +189,53 @@ def test_forward_rejects_host_only_layout(lib):
     assert ei.value.status == 1
     lay.close()
     bsa.bsa_free(0)   # NULL is a no-op
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "bsa.h"
+
+int main(void) {
+  bsa_pattern spec = {0};
+  bsa_layout* lay = NULL;
+  const int32_t* row_ptr = NULL;
+  const int32_t* col_idx = NULL;
+  int rows = 0, nnz = 0, i;
+  spec.kind = BSA_PATTERN_BAND_GLOBAL;
+  spec.window = 1;
+  spec.global_first = 1;
+  if (bsa_build_layout(&spec, 256, 64, 1, -1, &lay) != BSA_OK) {
+    printf("build: %s\n", bsa_last_error());
+    return 1;
+  }
+  if (bsa_layout_csr(lay, &row_ptr, &col_idx, &rows, &nnz) != BSA_OK) return 2;
+  printf("%d %d", rows, nnz);
+  for (i = 0; i < nnz; ++i) printf(" %d", (int)col_idx[i]);
+  printf("\n");
+  /* a host-only layout is refused before anything is launched */
+  printf("%d\n", bsa_forward(NULL, NULL, NULL, lay, 64, 256, 1, 1, 64, 0.125f, NULL, NULL, NULL) != BSA_OK);
+  bsa_free(lay);
+  bsa_free(NULL);
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/bsa.h compiles as C99 with warnings as errors, and a C program
+    linked against libbsa.so builds a host-only layout: the 4-block band
+    layout with block 0 has rows {0}, {0,1}, {0,1,2}, {0,2,3}."""
+    import shutil
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(bsa.LIB_PATH)
+    inc = os.path.join(os.path.dirname(libdir), "include")
+    res = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", f"-I{inc}", str(src), "-o", str(exe),
+                          f"-L{libdir}", "-lbsa", f"-Wl,-rpath,{libdir}"], capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert run.stdout.split("\n")[:2] == ["4 9 0 0 1 0 1 2 0 2 3", "1"]
