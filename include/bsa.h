@@ -174,7 +174,10 @@ int bsa_debug_timeout_probe(const bsa_layout* layout, int d, uint64_t timeout_ns
  * synchronising `stream` makes o_host and lse_host valid.  Layouts and
  * requirements as for bsa_forward, plus host pointers non-null (page-locked
  * host memory lets the copies overlap; pageable memory works but serialises
- * them) and groups >= 1.  No device allocation. */
+ * them) and groups >= 1; these are checked before anything is enqueued.  A
+ * CUDA error while enqueueing (not expected) returns BSA_ERR_CUDA with the
+ * runs before it already enqueued; synchronise the device before reusing the
+ * buffers then.  No device allocation. */
 int bsa_forward_host(const void* q_host, const void* k_host, const void* v_host,
                      const bsa_layout* layout, int B, int n, int heads, int kv_heads,
                      int d, float scale, void* q, void* k, void* v, void* o, float* lse,
