@@ -239,3 +239,45 @@ def test_header_is_plain_c_and_links(tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0, run.stdout + run.stderr
     assert run.stdout.split("\n")[:2] == ["4 9 0 0 1 0 1 2 0 2 3", "1"]
+
+
+def test_random_specs_bit_exact_sweep(lib):
+    """A seeded sweep over every pattern family's parameters (sizes, ragged
+    ends, block sizes, layout heads, windows, dyadic exponents, densities,
+    seeds and explicit masks): CSR, longest-first order, transposed layout
+    and gradient segments all equal the oracle's rules."""
+    rng = np.random.default_rng(2024)
+    for trial in range(40):
+        kind = [OL.BAND_GLOBAL, OL.DYADIC, OL.RANDOM, OL.EXPLICIT][trial % 4]
+        B = int(rng.choice([64, 128]))
+        n = int(rng.integers(1, 40 * B))
+        L = int(rng.integers(1, 4))
+        nb = OL.n_blocks(n, B)
+        if kind == OL.BAND_GLOBAL:
+            kw = dict(window=int(rng.integers(0, 6)), global_first=int(rng.integers(0, 2)))
+        elif kind == OL.DYADIC:
+            kw = dict(window=int(rng.integers(0, 4)), global_first=int(rng.integers(0, 2)),
+                      dyadic_kmin=int(rng.integers(0, 5)))
+        elif kind == OL.RANDOM:
+            kw = dict(density=float(rng.random()), seed=int(rng.integers(0, 2 ** 63)))
+        else:
+            mask = (rng.random((L, nb, nb)) < rng.random()) & np.tri(nb, dtype=bool)[None]
+            kw = dict(mask=mask.astype(np.uint8))
+        okw = dict(kw, mask=kw["mask"].astype(bool).tolist()) if kind == OL.EXPLICIT else kw
+        rp, ci, order = _csr_from_lib(kind, n, B, L, **kw)
+        sets = OL.kept_sets(kind, n, B, L, **okw)
+        orp, oci = OL.to_csr(sets)
+        label = f"trial {trial}: kind {kind} n {n} B {B} L {L} {kw if kind != OL.EXPLICIT else ''}"
+        np.testing.assert_array_equal(rp, np.array(orp, dtype=np.int32), err_msg=label)
+        np.testing.assert_array_equal(ci, np.array(oci, dtype=np.int32), err_msg=label)
+        _check_order(rp, order, L, nb)
+        lay = bsa.Layout(kind, n, B, L, -1, **kw)
+        cp, ri = bsa.bsa_layout_csc(lay.handle)
+        seg_ptr, segs = bsa.bsa_layout_segments(lay.handle)
+        lay.close()
+        ocp, ori = OL.to_csc(sets)
+        np.testing.assert_array_equal(cp, np.array(ocp, dtype=np.int32), err_msg=label)
+        np.testing.assert_array_equal(ri, np.array(ori, dtype=np.int32), err_msg=label)
+        want_ptr, want = _segments_from_csc(ocp, L, nb)
+        np.testing.assert_array_equal(seg_ptr, want_ptr, err_msg=label)
+        np.testing.assert_array_equal(segs.reshape(-1, 3), want, err_msg=label)
