@@ -165,3 +165,76 @@ def test_p4_arithmetic(golden_dir):
     # the dense causal token-pair count the BF1 ratio divides into
     sets = L.kept_sets(L.BAND_GLOBAL, 1024, 64, 1, window=10 ** 6, global_first=1)[0]
     assert L.kept_token_pairs(sets, 1024, 64) == 1024 * 1025 // 2
+
+
+# ------------------------------------------------------------ transposed layout
+def _csc_columns(sets_one_head):
+    col_ptr, row_idx = L.to_csc([sets_one_head])
+    return [row_idx[col_ptr[j]:col_ptr[j + 1]] for j in range(len(col_ptr) - 1)]
+
+
+def test_csc_hand_derived_columns(golden_dir):
+    """The tiny band workload's columns, read off its rows by hand."""
+    g = _load(golden_dir, "layout_rows.json")
+    case = g["cases"][0]
+    sets = L.kept_sets(case["kind"], case["n"], case["B"], 1, window=case["window"],
+                       global_first=case["global_first"])[0]
+    assert _csc_columns(sets) == case["cols"]
+
+
+@pytest.mark.parametrize("nb,window,global_first", [(40, 2, 1), (33, 0, 0), (17, 5, 1), (9, 0, 1)])
+def test_csc_band_closed_form(nb, window, global_first):
+    """Inverting the band rule: key block j > 0 is kept by the query blocks
+    j .. j + window (those inside the sequence); block 0 by the first window + 1
+    blocks, or by every block when the global first block is kept."""
+    sets = L.kept_sets(L.BAND_GLOBAL, nb * 64, 64, 1, window=window, global_first=global_first)[0]
+    cols = _csc_columns(sets)
+    for j in range(nb):
+        if j == 0 and global_first:
+            want = list(range(nb))
+        else:
+            want = list(range(j, min(nb, j + window + 1)))
+        assert cols[j] == want, j
+
+
+def test_csc_dyadic_closed_form():
+    """Inverting BF1's route ("BF1 ...", Method, section 3.1): key block j > 0
+    is kept by i = j, j + 1, j + 2 (self and the two local predecessors) and by
+    i = j + 2^k for k >= 2; block 0 by every query block."""
+    nb = 512
+    sets = L.kept_sets(L.DYADIC, nb * 64, 64, 1, window=2, global_first=1, dyadic_kmin=2)[0]
+    cols = _csc_columns(sets)
+    assert cols[0] == list(range(nb))
+    for j in range(1, nb):
+        want = {j, j + 1, j + 2} | {j + (1 << k) for k in range(2, 10)}
+        assert cols[j] == sorted(i for i in want if i < nb), j
+
+
+@pytest.mark.parametrize("kind,kw", [
+    (L.BAND_GLOBAL, dict(window=3, global_first=1)),
+    (L.DYADIC, dict(window=2, global_first=1, dyadic_kmin=2)),
+    (L.RANDOM, dict(density=0.3, seed=11)),
+])
+def test_csc_is_the_transposed_block_mask(kind, kw):
+    """Columns of the transposed layout equal the nonzero rows of each column
+    of the dense block mask M_B, transposed by numpy, for every layout head."""
+    np = pytest.importorskip("numpy")
+    sets = L.kept_sets(kind, 37 * 64, 64, 2, **kw)
+    col_ptr, row_idx = L.to_csc(sets)
+    nb = 37
+    for h in range(2):
+        mt = np.array(L.block_mask(sets[h]), dtype=np.uint8).T
+        for j in range(nb):
+            c = h * nb + j
+            assert row_idx[col_ptr[c]:col_ptr[c + 1]] == [int(i) for i in np.nonzero(mt[j])[0]]
+    assert col_ptr[-1] == sum(len(r) for s in sets for r in s)
+
+
+def test_csc_pins_catch_a_planted_transpose():
+    """A transposed layout built from the rows instead of the columns (the
+    mistake a shared misreading would make on both sides) fails the closed form."""
+    nb = 64
+    sets = L.kept_sets(L.DYADIC, nb * 64, 64, 1, window=2, global_first=1, dyadic_kmin=2)[0]
+    wrong = [sorted(sets[j]) for j in range(nb)]          # rows, not columns
+    want5 = sorted(i for i in {5, 6, 7} | {5 + (1 << k) for k in range(2, 6)} if i < nb)
+    assert wrong[5] != want5 and _csc_columns(sets)[5] == want5
