@@ -41,7 +41,11 @@ from block_sparse_long_bsa_b200.workloads import WORKLOADS, ORDER, HEADLINE  # n
 METRIC = "block-sparse attn fwd effective TFLOPS (4·d·kept pairs/s), % of B200 bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SRC = os.path.join(ROOT, "block_sparse_long_bsa_b200", "csrc", "bsa_fwd_sm100a.cu")
+CSRC = os.path.join(ROOT, "block_sparse_long_bsa_b200", "csrc")
+# every source the forward kernel is compiled or launched from: the kernel,
+# the device helpers it includes and the tensor-map encoding of its boxes
+KERNEL_SRCS = [os.path.join(CSRC, f) for f in
+               ("bsa_fwd_sm100a.cu", "bsa_device.cuh", "bsa_tmap.cpp", "bsa_tmap.h")]
 THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                  0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                  0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
@@ -91,8 +95,12 @@ def load_peaks():
 
 
 def kernel_sha():
-    with open(KERNEL_SRC, "rb") as fh:
-        return hashlib.sha256(fh.read()).hexdigest()
+    """sha256 over the forward kernel's sources, in a fixed order."""
+    h = hashlib.sha256()
+    for path in KERNEL_SRCS:
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 E2E_GROUPS = 8   # key/value-head runs of the end-to-end call

@@ -25,6 +25,9 @@ int set_error(int status, const std::string& msg) {
   g_last_error = msg;
   return status;
 }
+int counter_error(const char* what, cudaError_t e) {
+  return set_error(BSA_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
 }  // namespace bsa
 
 using bsa::set_error;
@@ -332,13 +335,23 @@ int bsa_debug_timeout_probe(const bsa_layout* layout, int d, uint64_t timeout_ns
 }
 
 int bsa_get_status(const bsa_layout* layout, void* stream) {
-  int st = check_device(layout);
-  if (st != BSA_OK) return st;
+  if (!layout) return set_error(BSA_ERR_INVALID_ARG, "layout is NULL");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* d_word = nullptr;
+  if (layout->device < 0) {
+    // a host-only layout: the status word of the allocation-free entry point's
+    // static block on the current device
+    const int st = bsa::noalloc_status_word(&d_word);
+    if (st != BSA_OK) return st;
+  } else {
+    const int st = check_device(layout);
+    if (st != BSA_OK) return st;
+    d_word = layout->d_status;
+  }
   uint32_t word = 0;
-  cudaError_t e = cudaMemcpyAsync(&word, layout->d_status, sizeof(word), cudaMemcpyDeviceToHost, s);
+  cudaError_t e = cudaMemcpyAsync(&word, d_word, sizeof(word), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(layout->d_status, 0, sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(d_word, 0, sizeof(uint32_t), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("status read: ") + cudaGetErrorString(e));
   if (word & bsa::kStatusTimeout)
@@ -354,6 +367,8 @@ void bsa_free(bsa_layout* layout) {
     int prev = -1;
     if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
     cudaSetDevice(layout->device);
+    for (cudaEvent_t& ev : layout->counter_event)
+      if (ev) cudaEventDestroy(ev);
     cudaFree(layout->d_base);
     if (prev >= 0 && prev != layout->device) cudaSetDevice(prev);
   }

@@ -44,6 +44,17 @@
 namespace bsa {
 namespace bwd {
 
+// The last CTA of a launch to finish puts the work counter back to zero for the
+// next launch that uses it (the dq and dk/dv kernels of one call share one
+// counter one after the other; launches on one counter are ordered by the host).
+__device__ __forceinline__ void release_counter(uint32_t* counter) {
+  __threadfence();
+  if (atomicAdd(counter + 1, 1u) == gridDim.x - 1) {
+    atomicExch(counter, 0u);
+    atomicExch(counter + 1, 0u);
+  }
+}
+
 using namespace ptx;
 
 
@@ -73,7 +84,8 @@ struct Params {
   float* dk;
   float* dv;
   uint32_t* status;
-  uint32_t* work_counter;   // next unclaimed item of the launched kernel (zeroed before its launch)
+  uint32_t* work_counter;   // [0]: next unclaimed item of the launched kernel, [1]: its CTAs done;
+                            // both zero at launch, set back to zero by the last CTA
   int n, nb, L, heads, kv_heads, group, pack, n_steps;   // n_steps = group / pack head steps per key/value head
   int items;         // work items of the launched kernel
   float scale, scale_log2;
@@ -646,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) release_counter(p.work_counter);
 }
 
 // ---------------------------------------------------------------- dK, dV
@@ -1006,6 +1019,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) release_counter(p.work_counter);
 }
 
 }  // namespace bwd
@@ -1087,15 +1101,10 @@ int launch_instance(const Launch& a, const bwd::Params& p) {
   bwd::Params pq = p, pk = p;
   pq.items = a.items_dq;
   pk.items = a.items_dkv;
-  // the two product kernels share one item counter, cleared before each
-  if (a.items_dq > 0) {
-    e = cudaMemsetAsync(pq.work_counter, 0, sizeof(uint32_t), a.stream);
-    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing the item counter: ") + cudaGetErrorString(e));
+  // the two product kernels share one item counter, one after the other
+  if (a.items_dq > 0)
     kq<<<a.items_dq < a.sms ? a.items_dq : a.sms, bwd::kThreads, smem_q, a.stream>>>(mq, mdo, mk2, mv2, pq);
-  }
   if (a.items_dkv > 0) {
-    e = cudaMemsetAsync(pk.work_counter, 0, sizeof(uint32_t), a.stream);
-    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing the item counter: ") + cudaGetErrorString(e));
     kkv<<<a.items_dkv < a.sms ? a.items_dkv : a.sms, bwd::kThreads, smem_kv, a.stream>>>(mq, mdo, mk, mv, pk);
   }
   e = cudaGetLastError();
@@ -1155,11 +1164,6 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   p.dk = dk;
   p.dv = dv;
   p.status = layout->d_status;
-  {
-    // one of the layout's work counters, taken in turn with its forwards
-    const uint32_t call = const_cast<bsa_layout*>(layout)->calls.fetch_add(1, std::memory_order_relaxed);
-    p.work_counter = layout->d_status + 64 + size_t(call % kWorkCounters) * 32;
-  }
   p.n = n;
   p.nb = layout->nb;
   p.L = layout->L;
@@ -1176,8 +1180,12 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   if (e != cudaSuccess || sms < 1) return set_error(BSA_ERR_CUDA, "cannot query the SM count");
   Launch a{q, k, v, o, dout, heads, kv_heads, n, int(items_dq), int(items_dkv), sms, size_t(heads) * n, workspace,
            static_cast<cudaStream_t>(stream)};
-  if (B == 64 && d == 128) return launch_instance<64, 128>(a, p);
-  if (B == 64 && d == 64) return launch_instance<64, 64>(a, p);
-  if (B == 128 && d == 128) return launch_instance<128, 128>(a, p);
-  return launch_instance<128, 64>(a, p);
+  // one of the layout's work counters, taken in turn with its forwards
+  return with_work_counter(layout, a.stream, [&](uint32_t* counter) {
+    p.work_counter = counter;
+    if (B == 64 && d == 128) return launch_instance<64, 128>(a, p);
+    if (B == 64 && d == 64) return launch_instance<64, 64>(a, p);
+    if (B == 128 && d == 128) return launch_instance<128, 128>(a, p);
+    return launch_instance<128, 64>(a, p);
+  });
 }

@@ -19,7 +19,7 @@
 //   O += P V_j                 (tcgen05.mma with A = P read from TMEM)
 // then o = O / l (bf16, stored row by row) and lse = (m + log2 l) * ln 2.
 // The running max is only moved when a block's max exceeds it by more than
-// 2^8 (in exp2 units), which keeps P <= 256 (exact in bf16's range) and skips
+// 8 in exp2 units (a factor of 2^8), which keeps P <= 256 and skips
 // almost every rescale of O; the final normalisation uses the same max as the
 // sum, so the result is the plain softmax.
 //
@@ -62,7 +62,8 @@ struct Params {
   __nv_bfloat16* o;
   float* lse;
   uint32_t* status;
-  uint32_t* work_counter;   // next unclaimed item of the longest-first list (zeroed before launch)
+  uint32_t* work_counter;   // [0]: next unclaimed item of the longest-first list, [1]: CTAs done;
+                            // both zero at launch, set back to zero by the last CTA
   int n, nb, heads, L, group;
   int items;         // work items in the longest-first list
   int pack;          // distinct heads per tile (1 or 2)
@@ -177,6 +178,16 @@ __device__ __forceinline__ void st_global_v4(void* ptr, const uint32_t* u) {
   asm volatile("st.global.v4.b32 [%0], {%1,%2,%3,%4};" ::"l"(ptr), "r"(u[0]), "r"(u[1]), "r"(u[2]),
                "r"(u[3])
                : "memory");
+}
+
+// The last CTA of a launch to finish puts the work counter back to zero for the
+// next launch that uses it (launches on one counter are ordered by the host).
+__device__ __forceinline__ void release_counter(uint32_t* counter) {
+  __threadfence();
+  if (atomicAdd(counter + 1, 1u) == gridDim.x - 1) {
+    atomicExch(counter, 0u);
+    atomicExch(counter + 1, 0u);
+  }
 }
 
 // Chunk c (counted over all items of the CTA) uses S buffer c & 1, K slot
@@ -662,6 +673,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     tc_fence_after();
     tmem_dealloc(tmem, S::kTmemCols);
   }
+  if (threadIdx.x == 0) release_counter(p.work_counter);
 }
 
 }  // namespace dev
@@ -714,10 +726,6 @@ int launch_instance(const ForwardArgs& a, dev::Params p) {
   } else {
     grid = 8;
   }
-  if (!a.debug_never) {
-    e = cudaMemsetAsync(p.work_counter, 0, sizeof(uint32_t), static_cast<cudaStream_t>(a.stream));
-    if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("clearing the work counter: ") + cudaGetErrorString(e));
-  }
   kern<<<grid, dev::kThreads, smem, static_cast<cudaStream_t>(a.stream)>>>(mq, mk, mv, mo, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
@@ -736,10 +744,6 @@ int launch_forward(const ForwardArgs& a) {
   p.order = L->d_order;
   p.lse = a.lse;
   p.status = L->d_status;
-  {
-    const uint32_t call = const_cast<bsa_layout*>(L)->calls.fetch_add(1, std::memory_order_relaxed);
-    p.work_counter = L->d_status + 64 + size_t(call % kWorkCounters) * 32;
-  }
   p.n = a.n;
   p.nb = L->nb;
   p.heads = a.heads;
@@ -752,11 +756,14 @@ int launch_forward(const ForwardArgs& a) {
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
-  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 2>(a, p);
-  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2>(a, p);
-  return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
+  return with_work_counter(L, static_cast<cudaStream_t>(a.stream), [&](uint32_t* counter) {
+    p.work_counter = counter;
+    if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 2>(a, p);
+    if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 2>(a, p);
+    if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2>(a, p);
+    if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2>(a, p);
+    return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
+  });
 }
 
 int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int32_t* col_idx,

@@ -26,8 +26,10 @@
 namespace {
 
 // Layout of the static scratch, in 32-bit words: word 0 is the kernel's status
-// word (cleared at every call); words from kLayoutBase on hold row_ptr,
-// col_idx and the longest-first order of the layout, back to back.
+// word (cleared at every call; bsa_get_status with a host-only layout reads
+// it), words 32 and 33 the kernel's work counter (left at zero by every
+// launch); words from kLayoutBase on hold row_ptr, col_idx and the
+// longest-first order of the layout, back to back.
 constexpr size_t kScratchWords = (size_t(4) << 20) / 4 + 64;   // 4 MiB of layout + 256 B head
 constexpr size_t kLayoutBase = 64;
 constexpr size_t kLayoutWordsMax = kScratchWords - kLayoutBase;
@@ -40,7 +42,9 @@ uint32_t* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the static scratch on the current device.  The symbol's
 // name in host code is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// once per device (with that device current) and cached for the life of the
+// process; after a cudaDeviceReset of that device the cached address is stale,
+// so this entry point must not be used on a device once it has been reset.
 int scratch_on_current_device(uint32_t** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -62,6 +66,10 @@ int scratch_on_current_device(uint32_t** out) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
+
+namespace bsa {
+int noalloc_status_word(uint32_t** out) { return scratch_on_current_device(out); }
+}  // namespace bsa
 
 extern "C" int bsa_forward_noalloc(const void* q, const void* k, const void* v,
                                    const bsa_layout* layout, int B, int n, int heads, int kv_heads,
@@ -88,10 +96,20 @@ extern "C" int bsa_forward_noalloc(const void* q, const void* k, const void* v,
                                         " (4 MiB): use bsa_forward with a device layout instead");
   if (int64_t(heads) * layout->nb > INT32_MAX) return set_error(BSA_ERR_SHAPE, "too many work items");
 
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // The layout is copied from the caller's host vectors while the call runs; a
+  // graph captured around that copy would read them again at every replay,
+  // after they may have been freed, so a capturing stream is refused.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  cudaError_t ce = cudaStreamIsCapturing(s, &cap);
+  if (ce != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("cudaStreamIsCapturing: ") + cudaGetErrorString(ce));
+  if (cap != cudaStreamCaptureStatusNone)
+    return set_error(BSA_ERR_UNSUPPORTED,
+                     "bsa_forward_noalloc copies the layout from host memory at every call and is refused "
+                     "on a capturing stream; capture bsa_forward with a device layout instead");
   uint32_t* scratch = nullptr;
   int st = scratch_on_current_device(&scratch);
   if (st != BSA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t* d_row_ptr = reinterpret_cast<int32_t*>(scratch + kLayoutBase);
   int32_t* d_col_idx = d_row_ptr + (rows + 1);
   int32_t* d_order = d_col_idx + layout->col_idx.size();

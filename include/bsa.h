@@ -137,19 +137,29 @@ int bsa_layout_csc(const bsa_layout* layout, const int32_t** col_ptr,
  * device; B in {64, 128}; d in {64, 128}; heads and kv_heads >= 1,
  * heads % kv_heads == 0, heads % layout_heads == 0; scale finite and > 0;
  * q, k, v, o non-null and 16-byte aligned; lse non-null and 4-byte aligned.
- * o and lse must not overlap the inputs.  Enqueues a 4-byte clear of a work
- * counter and one kernel; returns after enqueueing them.  Each call takes the
- * next of 64 work counters held in the layout's device block, so forwards
- * (and backwards) with the same layout may run at the same time on different
- * streams (up to 64 in flight at once).  A device-side wait that runs out (never expected)
- * makes the kernel return early and is reported by bsa_get_status. */
+ * o and lse must not overlap the inputs.  Enqueues one kernel and returns.
+ * Work counters: each call takes the next of 64 work counters held in the
+ * layout's device block (the kernel leaves it at zero when it ends), so
+ * forwards and backwards with the same layout may run at the same time on
+ * different streams.  A call that comes back to a counter makes its stream
+ * wait for the previous call on that counter (an event the library records
+ * after each call), so any number of calls may be in flight: beyond 64 the
+ * calls are ordered, never mixed.  A call made while `stream` is capturing a
+ * CUDA graph gets one of 192 further counters of its own for good (the
+ * captured launch replays on it; replays of one graph run one after another)
+ * and BSA_ERR_UNSUPPORTED once those are used up.  The layout is locked
+ * while a call enqueues its work, so calls from several host threads are
+ * safe.  A device-side wait that runs out (never expected) makes the kernel
+ * return early and is reported by bsa_get_status. */
 int bsa_forward(const void* q, const void* k, const void* v,
                 const bsa_layout* layout, int B, int n, int heads, int kv_heads,
                 int d, float scale, void* o, float* lse, void* stream);
 
 /* Synchronise `stream`, then read and clear the layout's device status word:
  * BSA_OK, or BSA_ERR_DEVICE_TIMEOUT if any forward on this layout since the
- * last call had a wait run out. */
+ * last call had a wait run out.  For a host-only layout (device = -1) the
+ * word read is the status of the most recent bsa_forward_noalloc call on the
+ * current device. */
 int bsa_get_status(const bsa_layout* layout, void* stream);
 
 /* Diagnostics: launch the forward kernel of this layout's shape in a mode
@@ -197,11 +207,15 @@ int bsa_forward_host(const void* q_host, const void* k_host, const void* v_host,
  * holds it until the process exits), clears the status word and launches the
  * same kernel.  A layout needing more than 1,048,576 32-bit words
  * (rows + 1 + nnz + rows) is rejected with BSA_ERR_SHAPE.  The first call on a
- * device looks up that block's device address (cudaGetSymbolAddress), so make
- * the first call on each device before any stream capture.  All calls share
- * the block and each overwrites what the last one left: calls that overlap on
- * the GPU race.  A device wait that runs out is recorded only in the shared
- * block, not reported by this entry point. */
+ * device looks up that block's device address (cudaGetSymbolAddress) and keeps
+ * it for the process, so make the first call on each device before any stream
+ * capture, and do not use this entry point on a device after a
+ * cudaDeviceReset of it.  The layout arrays are copied from host memory at
+ * every call, so a call on a stream that is capturing a CUDA graph is refused
+ * with BSA_ERR_UNSUPPORTED and enqueues nothing.  All calls share the block
+ * and each overwrites what the last one left: calls that overlap on the GPU
+ * race.  A device wait that runs out is recorded in the block's status word,
+ * which bsa_get_status reads when given the host-only layout. */
 int bsa_forward_noalloc(const void* q, const void* k, const void* v,
                         const bsa_layout* layout, int B, int n, int heads, int kv_heads,
                         int d, float scale, void* o, float* lse, void* stream);
@@ -258,11 +272,11 @@ int bsa_decode(const void* q, const void* k_cache, const void* v_cache,
  * bsa_forward (checked before launch; errors launch nothing), plus dout, dq,
  * dk, dv 16-byte aligned and workspace 4-byte aligned.  Enqueues the clear
  * of dk and dv (two memsets, or a kernel clearing only the rows that several
- * CTAs add into), a 4-byte clear of a work counter before each of the dq and
- * dk/dv kernels, and three kernels (D, dq, dk/dv) on the stream, and returns.
- * The work counter is the next of the layout's 64, taken in turn with its
- * forwards, so up to 64 forwards and backwards on one layout may be in
- * flight at once.  The dk/dv kernel adds its partial sums in fp32, so their
+ * CTAs add into) and three kernels (D, dq, dk/dv) on the stream, and
+ * returns.  The dq and dk/dv kernels share one work counter, taken as for
+ * bsa_forward (the same rotation, ordering and capture rules), so forwards
+ * and backwards on one layout may be in flight at once in any number.  The
+ * dk/dv kernel adds its partial sums in fp32, so their
  * summation order (and last bits) may differ from run to run.  A wait that
  * runs out is reported by bsa_get_status as for the forward. */
 int bsa_backward(const void* q, const void* k, const void* v, const void* o,

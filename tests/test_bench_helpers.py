@@ -45,3 +45,22 @@ def test_traffic_only_while_the_profile_matches_the_source(tmp_path, monkeypatch
     # no profile at all gives none
     os.remove(tmp_path / "profiles" / f"bsa_fwd_sm100a_{w}.md")
     assert bench.profiled_traffic(w) is None
+
+
+def test_kernel_hash_covers_the_device_helpers_and_tensor_maps(tmp_path, monkeypatch):
+    """A change to the included device helpers or to the tensor-map encoding
+    (box shapes) changes the hash, so a profile taken before it is not reused."""
+    import shutil
+    copies = []
+    for path in bench.KERNEL_SRCS:
+        dst = tmp_path / os.path.basename(path)
+        shutil.copy(path, dst)
+        copies.append(str(dst))
+    monkeypatch.setattr(bench, "KERNEL_SRCS", copies)
+    base = bench.kernel_sha()
+    for c in copies:
+        with open(c, "a") as fh:
+            fh.write("\n// edited\n")
+        changed = bench.kernel_sha()
+        assert changed != base, c
+        base = changed
