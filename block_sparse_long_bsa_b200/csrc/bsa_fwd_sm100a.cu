@@ -106,13 +106,15 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // B = 64, two for B = 128), so S is a 128 x 64 fp32 tile, two S buffers and the
 // O accumulator fit in 256 TMEM columns, and two CTAs share each SM.
 constexpr int kChunk = 64;
-constexpr int kKSlots = 2;   // K ring: K_c lives in slot c % 2
-constexpr int kVSlots = 3;   // V ring: V_c lives in slot c % 3
-constexpr int kODone = 3;    // PV_c completes o_done[c % 3]
 constexpr int kItemSlots = 8;  // items claimed by the producer, handed to the other roles
 
-template <int BLK, int HD>
+// K_c lives in K slot c % KS and V_c in V slot c % VS; PV_c completes
+// o_done[c % VS] (the V slot of chunk c frees when PV_c is done).
+template <int BLK, int HD, int KS, int VS>
 struct KernelShape {
+  static constexpr int kKSlots = KS;
+  static constexpr int kVSlots = VS;
+  static constexpr int kODone = VS;
   static constexpr int kCPB = BLK / kChunk;                  // chunks per kept block
   static constexpr int kSubs = kTileM / BLK;                 // query blocks stacked in the tile
   static constexpr int kAtoms = HD / 64;                     // 128-byte swizzle atoms along d
@@ -124,13 +126,15 @@ struct KernelShape {
   static constexpr int kOffV = kOffK + kKSlots * kTileBytes;
   static constexpr int kOffBar = kOffV + kVSlots * kTileBytes;
   // barriers: q_full, q_free, k_full[2], v_full[3], s_full[2], p_full[2],
-  //           o_done[3], o_free, drain, never, stage_free, item_full[8]
-  static constexpr int kNumBars = 2 + kKSlots + kVSlots + 2 + 2 + kODone + 4 + kItemSlots;
+  //           o_done[VS], o_free, drain, never, item_full[8], k_free[KS],
+  //           stage_free[8]
+  static constexpr int kPend = 8;                            // producer's pending-staging FIFO
+  static constexpr int kNumBars = 2 + kKSlots + kVSlots + 2 + 2 + kODone + 3 + kItemSlots + kKSlots + kPend;
   static constexpr int kWarpStage = 32 * 128;                // one warp's 32 rows x 64 columns of o
   static_assert(4 * (HD / 64) * kWarpStage == 2 * kTileBytes, "o staging fills two V slots");
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kOffPend = kOffMisc + 16;             // producer's pending-staging FIFO
-  static constexpr int kOffItems = kOffPend + 32;            // claimed, decoded items, ring of 8
+  static constexpr int kOffPend = kOffMisc + 16;
+  static constexpr int kOffItems = kOffPend + 8 * kPend;     // claimed, decoded items, ring of 8
   static constexpr int kSmemUsed = kOffItems + 32 * kItemSlots;
   static constexpr int kColS = 0;                            // S buffers: columns 0..63, 64..127
   static constexpr int kColO = 2 * kChunk;
@@ -139,6 +143,10 @@ struct KernelShape {
   static constexpr uint32_t kIdescPV = idesc_bf16(kTileM, HD, 0, 1);
   static_assert(2 * kChunk + HD <= 256, "TMEM budget");
   static_assert(BLK == 64 || BLK == 128, "block size");
+  static_assert(KS >= 2 && VS >= 3, "the rings hold at least the two K and three V chunks of the issue order");
+  // at most VS items are waiting for their staging slots at any time
+  static_assert(VS <= kPend, "pending-staging FIFO");
+  static_assert(kSmemUsed <= 227 * 1024, "shared memory");
   static_assert(HD == 64 || HD == 128, "head dim");
 };
 
@@ -191,20 +199,23 @@ __device__ __forceinline__ void release_counter(uint32_t* counter) {
 }
 
 // Chunk c (counted over all items of the CTA) uses S buffer c & 1, K slot
-// c % 2 and V slot c % 3.  MMAs are issued in the order QK_0, QK_1, PV_0,
+// c % KS and V slot c % VS.  MMAs are issued in the order QK_0, QK_1, PV_0,
 // QK_2, PV_1, ..., and the producer loads in the same order (K_{q+1} before
-// V_q).  A K slot frees when QK_{c-2} completes (s_full of that buffer), a V
-// slot when PV_{c-3} completes (o_done[c % 3]).  Each such barrier completes
+// V_q).  A K slot frees when QK_{c-KS} completes (k_free[c % KS]), a V
+// slot when PV_{c-VS} completes (o_done[c % VS]).  Each such barrier completes
 // once per product of its residue class, and the load that waits on it is
 // the one the next product of that class needs, so a parity wait can be
 // neither one phase early nor two phases late.
-template <int BLK, int HD, int MIN_CTAS>
+template <int BLK, int HD, int MIN_CTAS, int KS, int VS>
 __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                    const Params p) {
-  using S = KernelShape<BLK, HD>;
+  using S = KernelShape<BLK, HD, KS, VS>;
   constexpr int CPB = S::kCPB;
+  constexpr int kKSlots = S::kKSlots;
+  constexpr int kVSlots = S::kVSlots;
+  constexpr int kODone = S::kODone;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t base = smem_addr(smem_raw);
   if (base & 1023u) {
@@ -229,12 +240,21 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   const uint32_t bOFree = bODone0 + 8u * kODone;
   const uint32_t bDrain = bOFree + 8u;
   const uint32_t bNever = bOFree + 16u;
-  // The epilogue of an item stages o in the V slots of its last two chunks
-  // (free once its last PV is done); stage_free completes when the TMA stores
-  // out of them have read them, once per item with at least one chunk.
-  const uint32_t bStageFree = bOFree + 24u;
-  const uint32_t bItemFull0 = bOFree + 32u;
+  const uint32_t bItemFull0 = bOFree + 24u;
   auto bItemFull = [&](int k) { return bItemFull0 + 8u * (k % kItemSlots); };
+  // k_free[s] completes when the QK^T that read K slot s has finished
+  const uint32_t bKFree0 = bItemFull0 + 8u * kItemSlots;
+  auto bKFree = [&](int c) { return bKFree0 + 8u * (c % kKSlots); };
+  // The epilogue of an item stages o in the V slots of its last two chunks
+  // (free once its last PV is done); stage_free[e % 8] completes when the TMA
+  // stores out of them have read them, e counting the items with at least one
+  // chunk.  Eight barriers in turn: the producer waits for item e only when a
+  // V load reaches its slots, at most VS - 1 <= 7 chunks after its last one,
+  // and eight later items (at least one chunk each) cannot all finish in that
+  // span, so the wait never sees its barrier two phases on.
+  const uint32_t bStageFree0 = bKFree0 + 8u * kKSlots;
+  auto bStageFree = [&](int e) { return bStageFree0 + 8u * (e % S::kPend); };
+  auto parStage = [](int e) { return uint32_t(e / S::kPend) & 1u; };
   // slot k % 8: {valid, row, start, len, h0, kvh, diag_last}
   volatile int* item_ring = reinterpret_cast<volatile int*>(gbase + S::kOffItems);
   auto read_item = [&](int k, Item& it) -> bool {
@@ -280,8 +300,9 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     mbar_init(bOFree, 128);
     mbar_init(bDrain, 1);
     mbar_init(bNever, 1);
-    mbar_init(bStageFree, 4);
+    for (int s = 0; s < S::kPend; ++s) mbar_init(bStageFree0 + 8u * s, 4);
     for (int s = 0; s < kItemSlots; ++s) mbar_init(bItemFull0 + 8u * s, 1);
+    for (int s = 0; s < kKSlots; ++s) mbar_init(bKFree0 + 8u * s, 1);
     *abort_flag = 0;
     fence_barrier_init();
     if (!p.debug_never) {
@@ -309,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       // Items with chunks whose staging slots the producer has not yet seen
       // freed: (ordinal among items with chunks, global index of last chunk).
       int* pend_ord = reinterpret_cast<int*>(gbase + S::kOffPend);
-      int* pend_last = pend_ord + 4;
+      int* pend_last = pend_ord + S::kPend;
       int pend_head = 0, pend_tail = 0, n_nonempty = 0;
       bool ok = true;
       if (p.debug_never) ok = ctl.wait(bNever, 0);
@@ -338,14 +359,14 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         ++q_loads;
         const int nch = it.len * CPB;
         if (nch > 0) {
-          pend_ord[pend_tail & 3] = n_nonempty++;
-          pend_last[pend_tail & 3] = kc + nch - 1;
+          pend_ord[pend_tail % S::kPend] = n_nonempty++;
+          pend_last[pend_tail % S::kPend] = kc + nch - 1;
           ++pend_tail;
         }
         auto key0 = [&](int q) { return __ldg(p.col_idx + it.start + q / CPB) * BLK + (q % CPB) * kChunk; };
         auto load_k = [&](int q) -> bool {
           const int c = kc;
-          if (c >= kKSlots && !ctl.wait(bSFull(c), parS(c - kKSlots))) return false;
+          if (c >= kKSlots && !ctl.wait(bKFree(c), parK(c - kKSlots))) return false;
           const uint32_t dst = sK + (c % kKSlots) * S::kTileBytes;
           mbar_expect_tx(bKFull(c), S::kTileBytes);
           const int r0 = key0(q);
@@ -356,10 +377,11 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         auto load_v = [&](int q) -> bool {
           const int c = vc;
           if (c >= kVSlots && !ctl.wait(bODone(c), parO(c - kVSlots))) return false;
-          // V_c refills the slot of chunk c - 3; if that chunk or chunk c - 2
-          // was the last of an item, its epilogue staged o there.
-          while (pend_head != pend_tail && c >= pend_last[pend_head & 3] + 2) {
-            if (!ctl.wait(bStageFree, uint32_t(pend_ord[pend_head & 3]) & 1u)) return false;
+          // V_c refills the slot of chunk c - VS; if that chunk or the one
+          // after it was the last of an item, its epilogue staged o there.
+          while (pend_head != pend_tail && c >= pend_last[pend_head % S::kPend] + kVSlots - 1) {
+            const int e = pend_ord[pend_head % S::kPend];
+            if (!ctl.wait(bStageFree(e), parStage(e))) return false;
             ++pend_head;
           }
           const uint32_t dst = sV + (c % kVSlots) * S::kTileBytes;
@@ -406,6 +428,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             mma_ss(d, a, b, S::kIdescQK, kk > 0 ? 1u : 0u);
           }
           tc_commit(bSFull(c));
+          tc_commit(bKFree(c));
           if (q == nch - 1) tc_commit(bQFree);      // last reader of this Q tile
           return true;
         };
@@ -459,6 +482,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     bool ok = true;
     int s_cnt = 0;                           // chunks seen (global chunk index base)
     bool stage_pending = false;              // this warp's last staging stores not yet released
+    int n_staged = 0;                        // items with at least one chunk staged so far
     // Once the TMA stores of the previous epilogue have read the staging box,
     // tell the producer (one arrival per warp); deferred so the store drains
     // while this warp already works on the next item.
@@ -466,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       if (stage_pending) {
         if (lane == 0) {
           asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-          mbar_arrive(bStageFree);
+          mbar_arrive(bStageFree(n_staged - 1));
         }
         __syncwarp();
         stage_pending = false;
@@ -646,6 +670,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         }
         if (lane == 0) asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         stage_pending = true;
+        ++n_staged;
       } else {
         // an item without kept blocks: o = 0 (rare; plain stores)
         if (sub < p.pack && tok < p.n && !*abort_flag) {
@@ -683,10 +708,10 @@ namespace {
 
 using namespace tmap;
 
-template <int BLK, int HD, int MIN_CTAS>
+template <int BLK, int HD, int MIN_CTAS, int KS = 2, int VS = 3>
 int launch_instance(const ForwardArgs& a, dev::Params p) {
-  using S = dev::KernelShape<BLK, HD>;
-  auto kern = dev::bsa_fwd_kernel<BLK, HD, MIN_CTAS>;
+  using S = dev::KernelShape<BLK, HD, KS, VS>;
+  auto kern = dev::bsa_fwd_kernel<BLK, HD, MIN_CTAS, KS, VS>;
   // Ask for enough shared memory that no more than MIN_CTAS CTAs share an SM,
   // so every resident CTA's TMEM allocation succeeds at once.
   int smem = S::kSmemUsed;
@@ -732,6 +757,15 @@ int launch_instance(const ForwardArgs& a, dev::Params p) {
   return BSA_OK;
 }
 
+// The kernel instance for (B, d): CTAs per SM and the depth of the K and V rings.
+int launch_shape(const ForwardArgs& a, const dev::Params& p) {
+  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 2>(a, p);
+  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 2>(a, p);
+  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2>(a, p);
+  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2>(a, p);
+  return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
+}
+
 }  // namespace
 
 int launch_forward(const ForwardArgs& a) {
@@ -758,11 +792,7 @@ int launch_forward(const ForwardArgs& a) {
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
   return with_work_counter(L, static_cast<cudaStream_t>(a.stream), [&](uint32_t* counter) {
     p.work_counter = counter;
-    if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 2>(a, p);
-    if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 2>(a, p);
-    if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2>(a, p);
-    if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2>(a, p);
-    return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
+    return launch_shape(a, p);
   });
 }
 
@@ -790,11 +820,7 @@ int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int3
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.items = (a.heads / p.pack) * L->nb;
   if (p.items < 1) return set_error(BSA_ERR_SHAPE, "no work items");
-  if (a.B == 128 && a.d == 128) return launch_instance<128, 128, 2>(a, p);
-  if (a.B == 128 && a.d == 64) return launch_instance<128, 64, 2>(a, p);
-  if (a.B == 64 && a.d == 128) return launch_instance<64, 128, 2>(a, p);
-  if (a.B == 64 && a.d == 64) return launch_instance<64, 64, 2>(a, p);
-  return set_error(BSA_ERR_UNSUPPORTED, "unsupported (B, d)");
+  return launch_shape(a, p);
 }
 
 }  // namespace bsa

@@ -46,3 +46,16 @@ def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
 
 def default_scale(d):
     return 1.0 / math.sqrt(d)
+
+
+def bf16_half_ulp(x):
+    """Half the gap between neighbouring bf16 numbers at each value x (x itself
+    a bf16 number): the most that rounding to nearest can have moved a real
+    number whose rounded value is x.  bf16 keeps 8 significant bits, so for
+    2^(e-1) <= |x| < 2^e the gap is 2^(e-8) and half of it 2^(e-9).  (A value
+    just below 2^e that rounds up to 2^e moves by at most half the smaller gap
+    below it, which is inside this bound too.)  Zero gets the bound of the
+    smallest subnormal, 2^-134."""
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    _, e = np.frexp(x)          # x = f 2^e with 1/2 <= f < 1
+    return np.where(x > 0, np.ldexp(1.0, e - 9), 2.0 ** -134)

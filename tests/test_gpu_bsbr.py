@@ -6,11 +6,19 @@ grouped-query heads and ragged ends.
 
 Tolerance.  The retrieval is computed with fp32 sums, exact bf16 x bf16
 products and a state split into bf16 hi + lo parts (relative error about
-2^-16), so its error is dominated by the final rounding of o to bf16
-(relative error up to 2^-8, bf16's unit roundoff with 8 significant bits).  The summed output adds the within-chunk term's own error
-(the forward's 1e-2 bound) and the rounding of that term to bf16 before the
-add.  Elementwise: |o - o_ref| <= 1.5e-2 + 2^-8 |o_ref| for the sum and
-<= 2^-8 |ref| + 1e-4 max |ref| for the retrieval term alone.
+2^-16), and the result is rounded to bf16 once.  That rounding moves a value
+by at most half the gap between bf16 neighbours at the rounded value
+(``bf16_half_ulp``, a property of round-to-nearest, pinned on the CPU), so
+each bound is that allowance plus an arithmetic budget, and only the
+arithmetic can use up the budget, never the luck of where a value falls
+between two bf16 numbers:
+  retrieval term alone:  |o - o_ref| <= half_ulp(o) + 1e-4 max |ref|
+  summed output:         |o - o_ref| <= half_ulp(o) + 1.5e-2
+(the within-chunk term's own 1e-2 bound, its rounding to bf16 before the
+add, and the retrieval's arithmetic).  Both are tighter than the relative
+2^-8 |ref| allowance they replace, which equals half_ulp only at the bottom
+of each binade.  Each test prints the worst share of its bound and the
+worst share of the arithmetic budget left after the rounding allowance.
 """
 import math
 
@@ -25,7 +33,7 @@ from oracle import attention as OA
 from oracle import bsbr as BS
 from oracle import layouts as OL
 
-from gpu_common import to_device_bf16
+from gpu_common import bf16_half_ulp, to_device_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -78,9 +86,11 @@ def test_retrieval_term_alone(case):
     got = o.float().cpu().numpy()
     assert np.all(got[:, :B] == 0)
     err = np.abs(got - ref)
-    bound = 2.0 ** -8 * np.abs(ref) + 1e-4 * np.abs(ref).max()
+    budget = 1e-4 * np.abs(ref).max()
+    bound = bf16_half_ulp(got) + budget
     print(f"retrieval h{heads}/{kv} n{n} d{d} B{B}: max {err.max():.3e} (max |ref| {np.abs(ref).max():.2f}), "
-          f"worst ratio {(err / bound).max():.3f}")
+          f"worst share of bound {(err / bound).max():.3f}, "
+          f"of arithmetic budget {((err - bf16_half_ulp(got)) / budget).max():.3f}")
     assert np.all(err <= bound)
     lay.close()
 
@@ -98,9 +108,10 @@ def test_bsbr_output(case):
     ref = o_in + BS.retrieval(qh, kh, vh, B, scale)
     got = o.float().cpu().numpy()
     err = np.abs(got - ref)
-    bound = 1.5e-2 + 2.0 ** -8 * np.abs(ref)
+    bound = bf16_half_ulp(got) + 1.5e-2
     print(f"bsbr h{heads}/{kv} n{n} d{d} B{B}: max {err.max():.3e} mean {err.mean():.3e}, "
-          f"worst ratio {(err / bound).max():.3f}")
+          f"worst share of bound {(err / bound).max():.3f}, "
+          f"of arithmetic budget {((err - bf16_half_ulp(got)) / 1.5e-2).max():.3f}")
     assert np.all(err <= bound)
     assert err.mean() <= 1e-3 + 2.0 ** -9 * np.abs(ref).mean()
     assert np.abs(lse.cpu().numpy() - lse_ref).max() <= 1e-2
