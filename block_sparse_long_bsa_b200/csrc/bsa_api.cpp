@@ -98,7 +98,9 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     const size_t b_sp = lay->seg_ptr.size() * sizeof(int32_t);
     const size_t b_sg = std::max<size_t>(1, lay->segs.size()) * sizeof(int32_t);
     const size_t o_sp = o_ri + round_up(b_ri, 256), o_sg = o_sp + round_up(b_sp, 256);
-    const size_t o_st = o_sg + round_up(b_sg, 256), total = o_st + bsa::kStatusBlockBytes;
+    const size_t b_wk = lay->work.size() * sizeof(int32_t);
+    const size_t o_wk = o_sg + round_up(b_sg, 256);
+    const size_t o_st = o_wk + round_up(b_wk, 256), total = o_st + bsa::kStatusBlockBytes;
     void* base = nullptr;
     e = cudaMalloc(&base, total);
     if (e != cudaSuccess) {
@@ -121,6 +123,7 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     if (e == cudaSuccess) e = cudaMemcpy(c + o_sp, lay->seg_ptr.data(), b_sp, cudaMemcpyHostToDevice);
     if (e == cudaSuccess && !lay->segs.empty())
       e = cudaMemcpy(c + o_sg, lay->segs.data(), lay->segs.size() * sizeof(int32_t), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(c + o_wk, lay->work.data(), b_wk, cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemset(c + o_st, 0, bsa::kStatusBlockBytes);
     if (e != cudaSuccess) {
       cudaFree(base);
@@ -136,6 +139,7 @@ int bsa_build_layout(const bsa_pattern* spec, int n, int B, int layout_heads, in
     lay->d_row_idx = reinterpret_cast<const int32_t*>(c + o_ri);
     lay->d_seg_ptr = reinterpret_cast<const int32_t*>(c + o_sp);
     lay->d_segs = reinterpret_cast<const int32_t*>(c + o_sg);
+    lay->d_work = reinterpret_cast<const int32_t*>(c + o_wk);
     lay->d_status = reinterpret_cast<uint32_t*>(c + o_st);
     lay->device = device;
     if (prev >= 0 && prev != device) cudaSetDevice(prev);

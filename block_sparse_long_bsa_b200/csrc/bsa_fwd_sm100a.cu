@@ -56,13 +56,12 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.693147180559945309f;
 
 struct Params {
-  const int32_t* row_ptr;
+  const int4* work;            // per (layout head, rank): {query block, first CSR entry, kept blocks, diagonal last}
   const int32_t* col_idx;
-  const int32_t* order;
   __nv_bfloat16* o;
   float* lse;
   uint32_t* status;
-  uint32_t* work_counter;   // [0]: next unclaimed item of the longest-first list, [1]: CTAs done;
+  uint32_t* work_counter;   // [0]: items claimed beyond the first one of each CTA, [1]: CTAs done;
                             // both zero at launch, set back to zero by the last CTA
   int n, nb, heads, L, group;
   int items;         // work items in the longest-first list
@@ -156,29 +155,38 @@ struct Item {
   bool diag_last;
 };
 
-__device__ __forceinline__ Item decode_item(const Params& p, int t) {
-  Item it;
+// The work-table entry of item t (one 16-byte load; the producer issues it
+// for the next item while the current one is still loading).
+__device__ __forceinline__ int4 load_work(const Params& p, int t) {
   const int hg = t / p.nb;
   const int rank = t - hg * p.nb;
-  it.h0 = hg * p.pack;
+  const int lh = (hg * p.pack) % p.L;
+  return __ldg(p.work + size_t(lh) * p.nb + rank);
+}
+
+__device__ __forceinline__ Item decode_item(const Params& p, int t, int4 w) {
+  Item it;
+  it.h0 = (t / p.nb) * p.pack;
   it.kvh = it.h0 / p.group;
-  const int lh = it.h0 % p.L;
-  it.row = __ldg(p.order + size_t(lh) * p.nb + rank);
-  const size_t r = size_t(lh) * p.nb + it.row;
-  it.start = __ldg(p.row_ptr + r);
-  it.len = __ldg(p.row_ptr + r + 1) - it.start;
-  it.diag_last = it.len > 0 && __ldg(p.col_idx + it.start + it.len - 1) == it.row;
+  it.row = w.x;
+  it.start = w.y;
+  it.len = w.z;
+  it.diag_last = w.w != 0;
   return it;
 }
 
-// Persistent schedule: the producer of each CTA claims the next unclaimed
-// item of the longest-first list with one atomic add (greedy list
+// Persistent schedule: CTA b starts with item b of the longest-first list
+// (no atomic on the way to its first loads); after that the producer of each
+// CTA claims the next unclaimed item with one atomic add (greedy list
 // scheduling, so every CTA ends within about one item of the others) and
 // hands its index to the MMA and softmax roles through a ring of slots in
 // shared memory; -1 ends the stream.
+__device__ __forceinline__ int first_item(int n_items) {
+  return int(blockIdx.x) < n_items ? int(blockIdx.x) : -1;
+}
 __device__ __forceinline__ int claim_item(const Params& p, int n_items) {
   if (n_items <= 0) return -1;
-  const int t = int(atomicAdd(p.work_counter, 1u));
+  const int t = int(gridDim.x) + int(atomicAdd(p.work_counter, 1u));
   return t < n_items ? t : -1;
 }
 
@@ -334,11 +342,12 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
       int pend_head = 0, pend_tail = 0, n_nonempty = 0;
       bool ok = true;
       if (p.debug_never) ok = ctl.wait(bNever, 0);
-      int next_t = ok ? claim_item(p, n_items) : -1;
+      int next_t = ok ? first_item(n_items) : -1;
+      int4 next_w = next_t >= 0 ? load_work(p, next_t) : make_int4(0, 0, 0, 0);
       for (int k = 0; ok; ++k) {
         const int t = next_t;
         Item it{};
-        if (t >= 0) it = decode_item(p, t);
+        if (t >= 0) it = decode_item(p, t, next_w);
         volatile int* e = item_ring + 8 * (k % kItemSlots);
         e[0] = t >= 0;
         e[1] = it.row;
@@ -392,6 +401,9 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           return true;
         };
         if (nch > 0) ok = load_k(0);
+        // the claim above has returned by now: fetch the next item's entry
+        // while this item's loads wait for their slots
+        if (next_t >= 0) next_w = load_work(p, next_t);
         for (int q = 0; q < nch && ok; ++q) {
           if (q + 1 < nch) ok = load_k(q + 1);
           if (ok) ok = load_v(q);
@@ -773,9 +785,8 @@ int launch_forward(const ForwardArgs& a) {
   if (st != BSA_OK) return st;
   const bsa_layout* L = a.layout;
   dev::Params p{};
-  p.row_ptr = L->d_row_ptr;
+  p.work = reinterpret_cast<const int4*>(L->d_work);
   p.col_idx = L->d_col_idx;
-  p.order = L->d_order;
   p.lse = a.lse;
   p.status = L->d_status;
   p.n = a.n;
@@ -796,15 +807,13 @@ int launch_forward(const ForwardArgs& a) {
   });
 }
 
-int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int32_t* col_idx,
-                        const int32_t* order, uint32_t* status) {
+int launch_forward_with(const ForwardArgs& a, const int32_t* work, const int32_t* col_idx, uint32_t* status) {
   int st = get_encoder();
   if (st != BSA_OK) return st;
   const bsa_layout* L = a.layout;
   dev::Params p{};
-  p.row_ptr = row_ptr;
+  p.work = reinterpret_cast<const int4*>(work);
   p.col_idx = col_idx;
-  p.order = order;
   p.lse = a.lse;
   p.status = status;
   p.work_counter = status + kScratchCounterWord;

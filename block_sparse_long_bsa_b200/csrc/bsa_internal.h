@@ -33,6 +33,10 @@ struct bsa_layout {
   std::vector<int32_t> row_ptr;   // [L*nb + 1]
   std::vector<int32_t> col_idx;   // [nnz]
   std::vector<int32_t> order;     // [L*nb], longest row first per layout head
+  // [L*nb][4]: the forward's work table, per (layout head, rank in order):
+  // query block, first CSR entry, kept blocks, and 1 when the last kept block
+  // is the diagonal one, so one 16-byte load decodes a work item
+  std::vector<int32_t> work;
   std::vector<int32_t> col_ptr;   // [L*nb + 1]: transposed layout (CSC), per layout head
   std::vector<int32_t> row_idx;   // [nnz]: query blocks keeping each key block, ascending
   std::vector<int32_t> seg_ptr;   // [L + 1]: column segments of layout head h are seg_ptr[h] .. seg_ptr[h+1]
@@ -42,6 +46,7 @@ struct bsa_layout {
   const int32_t* d_row_ptr = nullptr;
   const int32_t* d_col_idx = nullptr;
   const int32_t* d_order = nullptr;
+  const int32_t* d_work = nullptr;   // 16-byte aligned
   const int32_t* d_col_ptr = nullptr;
   const int32_t* d_row_idx = nullptr;
   const int32_t* d_seg_ptr = nullptr;
@@ -61,7 +66,7 @@ namespace bsa {
 // Thread-local error message; returns the status for convenience.
 int set_error(int status, const std::string& msg);
 
-// Host layout compiler (bsa_layout.cpp).  Fills row_ptr/col_idx/order/max_row.
+// Host layout compiler (bsa_layout.cpp).  Fills row_ptr/col_idx/order/work/max_row.
 int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out);
 
 // Longest run of query blocks one key/value-gradient work item takes from a
@@ -106,10 +111,10 @@ struct ForwardArgs {
 
 int launch_forward(const ForwardArgs& a);
 
-// Same launch with the layout arrays and status word at explicit device
-// addresses (the allocation-free entry point stages them itself).
-int launch_forward_with(const ForwardArgs& a, const int32_t* row_ptr, const int32_t* col_idx,
-                        const int32_t* order, uint32_t* status);
+// Same launch with the forward's layout arrays (the work table, 16-byte
+// aligned, and col_idx) and the status word at explicit device addresses (the
+// allocation-free entry point stages them itself).
+int launch_forward_with(const ForwardArgs& a, const int32_t* work, const int32_t* col_idx, uint32_t* status);
 
 // Device address of the allocation-free entry point's status word on the
 // current device (bsa_noalloc.cu).

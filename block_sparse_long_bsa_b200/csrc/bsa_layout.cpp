@@ -201,6 +201,20 @@ int compile_layout(const bsa_pattern& spec, int n, int B, int L, bsa_layout* out
       return (rp[a + 1] - rp[a]) > (rp[b + 1] - rp[b]);
     });
   }
+  // The forward's work table: each (layout head, rank) decoded once here.
+  out->work.resize(size_t(4) * L * nb);
+  for (int h = 0; h < L; ++h) {
+    for (int rank = 0; rank < nb; ++rank) {
+      const int32_t row = out->order[size_t(h) * nb + rank];
+      const size_t r = size_t(h) * nb + row;
+      const int32_t start = out->row_ptr[r], len = out->row_ptr[r + 1] - start;
+      int32_t* w = out->work.data() + 4 * (size_t(h) * nb + rank);
+      w[0] = row;
+      w[1] = start;
+      w[2] = len;
+      w[3] = (len > 0 && out->col_idx[size_t(start) + len - 1] == row) ? 1 : 0;
+    }
+  }
   return BSA_OK;
 }
 

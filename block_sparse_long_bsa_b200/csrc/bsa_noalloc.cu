@@ -28,8 +28,9 @@ namespace {
 // Layout of the static scratch, in 32-bit words: word 0 is the kernel's status
 // word (cleared at every call; bsa_get_status with a host-only layout reads
 // it), words 32 and 33 the kernel's work counter (left at zero by every
-// launch); words from kLayoutBase on hold row_ptr, col_idx and the
-// longest-first order of the layout, back to back.
+// launch); words from kLayoutBase on (256 bytes in, so 16-byte aligned) hold
+// the layout's work table (four words per query block, longest row first)
+// and then col_idx.
 constexpr size_t kScratchWords = (size_t(4) << 20) / 4 + 64;   // 4 MiB of layout + 256 B head
 constexpr size_t kLayoutBase = 64;
 constexpr size_t kLayoutWordsMax = kScratchWords - kLayoutBase;
@@ -87,8 +88,7 @@ extern "C" int bsa_forward_noalloc(const void* q, const void* k, const void* v,
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
     return set_error(BSA_ERR_INVALID_ARG, "q, k, v and o must be 16-byte aligned");
   if (!aligned(lse, 4)) return set_error(BSA_ERR_INVALID_ARG, "lse must be 4-byte aligned");
-  const size_t rows = layout->row_ptr.size() - 1;
-  const size_t words = (rows + 1) + layout->col_idx.size() + layout->order.size();
+  const size_t words = layout->work.size() + layout->col_idx.size();
   if (words > kLayoutWordsMax)
     return set_error(BSA_ERR_SHAPE, "layout needs " + std::to_string(words) +
                                         " words of device scratch; the static scratch of this entry "
@@ -110,20 +110,16 @@ extern "C" int bsa_forward_noalloc(const void* q, const void* k, const void* v,
   uint32_t* scratch = nullptr;
   int st = scratch_on_current_device(&scratch);
   if (st != BSA_OK) return st;
-  int32_t* d_row_ptr = reinterpret_cast<int32_t*>(scratch + kLayoutBase);
-  int32_t* d_col_idx = d_row_ptr + (rows + 1);
-  int32_t* d_order = d_col_idx + layout->col_idx.size();
+  int32_t* d_work = reinterpret_cast<int32_t*>(scratch + kLayoutBase);
+  int32_t* d_col_idx = d_work + layout->work.size();
   cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(uint32_t), s);   // status word starts at zero
   if (e == cudaSuccess)
-    e = cudaMemcpyAsync(d_row_ptr, layout->row_ptr.data(), (rows + 1) * sizeof(int32_t),
+    e = cudaMemcpyAsync(d_work, layout->work.data(), layout->work.size() * sizeof(int32_t),
                         cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && !layout->col_idx.empty())
     e = cudaMemcpyAsync(d_col_idx, layout->col_idx.data(), layout->col_idx.size() * sizeof(int32_t),
                         cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(d_order, layout->order.data(), layout->order.size() * sizeof(int32_t),
-                        cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return set_error(BSA_ERR_CUDA, std::string("staging the layout: ") + cudaGetErrorString(e));
   bsa::ForwardArgs a{q, k, v, o, lse, layout, B, n, heads, kv_heads, d, scale, stream, 0, 0};
-  return bsa::launch_forward_with(a, d_row_ptr, d_col_idx, d_order, scratch);
+  return bsa::launch_forward_with(a, d_work, d_col_idx, scratch);
 }

@@ -201,12 +201,13 @@ int bsa_forward_host(const void* q_host, const void* k_host, const void* v_host,
  * while running, since cudaMalloc/cudaFree can synchronise the whole device.
  * Same arguments, checks and result as bsa_forward, except that `layout` may
  * be host-only (built with device = -1) and nothing is allocated: on the
- * caller's stream the call copies the layout's row_ptr, col_idx and order
- * arrays into a block of device memory that the library declares statically
- * (4 MiB of layout words plus a status word; every GPU that loads the library
- * holds it until the process exits), clears the status word and launches the
- * same kernel.  A layout needing more than 1,048,576 32-bit words
- * (rows + 1 + nnz + rows) is rejected with BSA_ERR_SHAPE.  The first call on a
+ * caller's stream the call copies what the kernel reads of the layout (its
+ * work table, four words per query block row, and col_idx) into a block of
+ * device memory that the library declares statically (4 MiB of layout words
+ * plus a status word; every GPU that loads the library holds it until the
+ * process exits), clears the status word and launches the same kernel.  A
+ * layout needing more than 1,048,576 32-bit words (4 * rows + nnz) is rejected
+ * with BSA_ERR_SHAPE.  The first call on a
  * device looks up that block's device address (cudaGetSymbolAddress) and keeps
  * it for the process, so make the first call on each device before any stream
  * capture, and do not use this entry point on a device after a

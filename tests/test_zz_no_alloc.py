@@ -103,7 +103,7 @@ def test_noalloc_refused_on_a_capturing_stream():
 
 
 def test_noalloc_refuses_layout_beyond_static_block():
-    # 400,000 one-block rows: row_ptr + col_idx + order need 1,200,001 words,
+    # 400,000 one-block rows: the work table and col_idx need 2,000,000 words,
     # more than the 1,048,576 the static block holds; refused before any copy
     n = 64 * 400_000
     big = bsa.Layout(OL.BAND_GLOBAL, n, 64, 1, -1, window=0, global_first=0)
