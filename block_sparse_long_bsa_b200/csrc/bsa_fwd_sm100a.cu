@@ -250,7 +250,11 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
   const uint32_t bNever = bOFree + 16u;
   const uint32_t bItemFull0 = bOFree + 24u;
   auto bItemFull = [&](int k) { return bItemFull0 + 8u * (k % kItemSlots); };
-  // k_free[s] completes when the QK^T that read K slot s has finished
+  // k_free[s] completes when the QK^T that read K slot s has finished.  With
+  // two K slots and two S buffers s_full of QK^T_c is already the completion
+  // of slot c % 2's reader, so the producer waits on it and QK^T commits
+  // nothing more (each commit costs tensor-pipe time).
+  constexpr bool kKFreeIsSFull = (kKSlots == 2);
   const uint32_t bKFree0 = bItemFull0 + 8u * kItemSlots;
   auto bKFree = [&](int c) { return bKFree0 + 8u * (c % kKSlots); };
   // The epilogue of an item stages o in the V slots of its last two chunks
@@ -375,7 +379,11 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
         auto key0 = [&](int q) { return __ldg(p.col_idx + it.start + q / CPB) * BLK + (q % CPB) * kChunk; };
         auto load_k = [&](int q) -> bool {
           const int c = kc;
-          if (c >= kKSlots && !ctl.wait(bKFree(c), parK(c - kKSlots))) return false;
+          if (c >= kKSlots) {
+            const bool freed = kKFreeIsSFull ? ctl.wait(bSFull(c), parS(c - kKSlots))
+                                             : ctl.wait(bKFree(c), parK(c - kKSlots));
+            if (!freed) return false;
+          }
           const uint32_t dst = sK + (c % kKSlots) * S::kTileBytes;
           mbar_expect_tx(bKFull(c), S::kTileBytes);
           const int r0 = key0(q);
@@ -440,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
             mma_ss(d, a, b, S::kIdescQK, kk > 0 ? 1u : 0u);
           }
           tc_commit(bSFull(c));
-          tc_commit(bKFree(c));
+          if constexpr (!kKFreeIsSFull) tc_commit(bKFree(c));
           if (q == nch - 1) tc_commit(bQFree);      // last reader of this Q tile
           return true;
         };
