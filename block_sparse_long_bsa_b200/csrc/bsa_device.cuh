@@ -263,6 +263,21 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo_bytes
   return d;
 }
 
+// The fields of sw128_desc other than the start address.  A descriptor is
+// these plus (address >> 4) in bits 0-13: shared-memory addresses stay below
+// 2^18, so a run-time base plus a tile offset never carries out of the field,
+// and an issuing loop can form each product's descriptors with one 32-bit add.
+__host__ __device__ constexpr uint64_t sw128_fixed(uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return (uint64_t((lbo_bytes >> 4) & 0x3FFFu) << 16) | (uint64_t((sbo_bytes >> 4) & 0x3FFFu) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// A descriptor from its low word (fixed bits plus address >> 4) and high word.
+__device__ __forceinline__ uint64_t desc_from(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
+}
+
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, shape
 // M x N; a_mn / b_mn = 1 for an operand stored along M / N (MN-major), 0 for
 // K-major.

@@ -427,6 +427,15 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
     if (lane == 0) {
       bool ok = true;
       int c0 = 0;            // chunks of earlier items (global chunk index base)
+      // Operand descriptors as fixed bits plus (address >> 4): each product
+      // adds its tile's offset to one of these low words.
+      constexpr uint64_t kFixKMajor = sw128_fixed(16, 1024);              // Q and K, read along d
+      constexpr uint64_t kFixV = sw128_fixed(S::kAtomRowsKV, 1024);       // V, read along the keys
+      const uint32_t q_lo = uint32_t(kFixKMajor) + (sQ >> 4);
+      const uint32_t k_lo = uint32_t(kFixKMajor) + (sK >> 4);
+      const uint32_t v_lo = uint32_t(kFixV) + (sV >> 4);
+      constexpr uint32_t kHiKMajor = uint32_t(kFixKMajor >> 32);
+      constexpr uint32_t kHiV = uint32_t(kFixV >> 32);
       if (p.debug_never) ok = ctl.wait(bNever, 0);
       for (int k = 0; ok; ++k) {
         if (!(ok = ctl.wait(bItemFull(k), uint32_t(k / kItemSlots) & 1u))) break;
@@ -440,11 +449,11 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           if (!ctl.wait(bKFull(c), parK(c))) return false;
           tc_fence_after();
           const uint32_t d = tmem + S::kColS + (c & 1) * kChunk;
-          const uint32_t kb = sK + (c % kKSlots) * S::kTileBytes;
+          const uint32_t kb_lo = k_lo + uint32_t(c % kKSlots) * (S::kTileBytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t a = sw128_desc(sQ + (kk >> 2) * S::kAtomRowsQ + (kk & 3) * 32, 16, 1024);
-            const uint64_t b = sw128_desc(kb + (kk >> 2) * S::kAtomRowsKV + (kk & 3) * 32, 16, 1024);
+            const uint64_t a = desc_from(q_lo + ((kk >> 2) * S::kAtomRowsQ + (kk & 3) * 32) / 16, kHiKMajor);
+            const uint64_t b = desc_from(kb_lo + ((kk >> 2) * S::kAtomRowsKV + (kk & 3) * 32) / 16, kHiKMajor);
             mma_ss(d, a, b, S::kIdescQK, kk > 0 ? 1u : 0u);
           }
           tc_commit(bSFull(c));
@@ -465,10 +474,10 @@ __global__ void __launch_bounds__(kThreads, MIN_CTAS)
           if (!ctl.wait(bPFull(c), parS(c))) return false;
           tc_fence_after();
           const uint32_t pa = tmem + S::kColS + (c & 1) * kChunk;
-          const uint32_t vb = sV + (c % kVSlots) * S::kTileBytes;
+          const uint32_t vb_lo = v_lo + uint32_t(c % kVSlots) * (S::kTileBytes >> 4);
 #pragma unroll
           for (int kk = 0; kk < kChunk / 16; ++kk) {
-            const uint64_t b = sw128_desc(vb + kk * 16 * 128, S::kAtomRowsKV, 1024);
+            const uint64_t b = desc_from(vb_lo + kk * 16 * 128 / 16, kHiV);
             mma_ts(tmem + S::kColO, pa + kk * 8, b, S::kIdescPV, (q > 0 || kk > 0) ? 1u : 0u);
           }
           tc_commit(bODone(c));
