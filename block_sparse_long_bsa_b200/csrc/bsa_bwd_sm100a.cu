@@ -479,7 +479,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
-          mma_ss(tmem + S::kColS, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
+          mma_ss(tmem + S::kColS, sw128<16, 1024>(qb + ao), sw128<16, 1024>(kb + bo), S::kIdescS, kk > 0);
         }
         tc_commit(bar(S::kBS));
       };
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
-          mma_ss(tmem + S::kColDP, sw128_desc(qb + ao, 16, 1024), sw128_desc(sV + bo, 16, 1024), S::kIdescS, kk > 0);
+          mma_ss(tmem + S::kColDP, sw128<16, 1024>(qb + ao), sw128<16, 1024>(sV + bo), S::kIdescS, kk > 0);
         }
         tc_commit(bar(S::kBDP));
         if (cs.c == dq_steps(cs.it) - 1) tc_commit(bar(S::kBQFree + (cs.xi & 1)));   // last reader of Q, dO
@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < S::kStep / 16; ++kk)
             mma_ts(acc, tmem + S::kColDP + (kk >> 2) * 64 + (kk & 3) * 8,
-                   sw128_desc(kb + kk * 16 * 128, S::kAtomKV, 1024), S::kIdescDQ, (cd.c > 0 || kk > 0) ? 1u : 0u);
+                   sw128<S::kAtomKV, 1024>(kb + kk * 16 * 128), S::kIdescDQ, (cd.c > 0 || kk > 0) ? 1u : 0u);
           tc_commit(bar(S::kBKFree + (cd.g & 1)));
           if (cd.c == dq_steps(cd.it) - 1) tc_commit(bar(S::kBAcc + (cd.xi & 1)));
         }
@@ -886,9 +886,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < kTileM / 16; ++kk) {
             const uint32_t off = kk * 16 * 128;
             const uint32_t acc = (cd.e > 0 || kk > 0) ? 1u : 0u;
-            mma_ss(accv, sw128_desc(qb + S::kQBytes + off, S::kAtomQ, 1024), sw128_desc(sP + off, S::kPBytes, 1024),
+            mma_ss(accv, sw128<S::kAtomQ, 1024>(qb + S::kQBytes + off), sw128<S::kPBytes, 1024>(sP + off),
                    S::kIdescT, acc);
-            mma_ss(acck, sw128_desc(qb + off, S::kAtomQ, 1024), sw128_desc(sDS + off, S::kPBytes, 1024), S::kIdescT,
+            mma_ss(acck, sw128<S::kAtomQ, 1024>(qb + off), sw128<S::kPBytes, 1024>(sDS + off), S::kIdescT,
                    acc);
           }
           tc_commit(bar(S::kBDone + (cd.t & 1)));
@@ -906,8 +906,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint32_t ao = (kk >> 2) * S::kAtomQ + (kk & 3) * 32, bo = (kk >> 2) * S::kAtomKV + (kk & 3) * 32;
-            mma_ss(ds, sw128_desc(qb + ao, 16, 1024), sw128_desc(kb + bo, 16, 1024), S::kIdescS, kk > 0);
-            mma_ss(ddp, sw128_desc(qb + S::kQBytes + ao, 16, 1024), sw128_desc(vb + bo, 16, 1024), S::kIdescS,
+            mma_ss(ds, sw128<16, 1024>(qb + ao), sw128<16, 1024>(kb + bo), S::kIdescS, kk > 0);
+            mma_ss(ddp, sw128<16, 1024>(qb + S::kQBytes + ao), sw128<16, 1024>(vb + bo), S::kIdescS,
                    kk > 0);
           }
           tc_commit(bar(S::kBS + (cs.t & 1)));

@@ -278,6 +278,14 @@ __device__ __forceinline__ uint64_t desc_from(uint32_t lo, uint32_t hi) {
   return d;
 }
 
+// sw128_desc with strides known at compile time: the shift of the address
+// and one 32-bit add form the low word; the high word is a constant.
+template <uint32_t LBO, uint32_t SBO>
+__device__ __forceinline__ uint64_t sw128(uint32_t addr) {
+  constexpr uint64_t kFix = sw128_fixed(LBO, SBO);
+  return desc_from(uint32_t(kFix) + (addr >> 4), uint32_t(kFix >> 32));
+}
+
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, shape
 // M x N; a_mn / b_mn = 1 for an operand stored along M / N (MN-major), 0 for
 // K-major.
