@@ -1,5 +1,5 @@
 """Shared helpers of the GPU parity tests: seeded inputs on the device, the
-oracle on the same bf16 bits, and the benchmark spec's tolerances."""
+oracle on the same bf16 bits, and the parity tolerances (max and mean absolute error)."""
 from __future__ import annotations
 
 import math
