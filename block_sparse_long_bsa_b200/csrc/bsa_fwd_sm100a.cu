@@ -209,8 +209,9 @@ __device__ __forceinline__ void release_counter(uint32_t* counter) {
 // Chunk c (counted over all items of the CTA) uses S buffer c & 1, K slot
 // c % KS and V slot c % VS.  MMAs are issued in the order QK_0, QK_1, PV_0,
 // QK_2, PV_1, ..., and the producer loads in the same order (K_{q+1} before
-// V_q).  A K slot frees when QK_{c-KS} completes (k_free[c % KS]), a V
-// slot when PV_{c-VS} completes (o_done[c % VS]).  Each such barrier completes
+// V_q).  A K slot frees when QK_{c-KS} completes (k_free[c % KS]; with two
+// K slots the s_full commit of that QK^T), a V slot when PV_{c-VS} completes
+// (o_done[c % VS]).  Each such barrier completes
 // once per product of its residue class, and the load that waits on it is
 // the one the next product of that class needs, so a parity wait can be
 // neither one phase early nor two phases late.
