@@ -2,9 +2,14 @@
 
 Element-by-element at sizes the oracle finishes in seconds (several tiles,
 ragged last blocks, every pattern family, packed and unpacked grouped-query
-tiles), and on sampled (head, query block) tiles of the full-size workloads in
-the launch configuration the benchmark times.  Tolerances: max |d| <= 1e-2 and
-mean |d| <= 1e-3 on o and lse; layouts bit-exact (checked on the CPU side).
+tiles), and at full size in the launch configuration the benchmark times:
+every head and block of the two 32K workloads, and two whole heads plus every
+head's longest rows of the 131K workload.  Also: future tokens and dropped
+blocks leave o bitwise unchanged, run-to-run bitwise determinism, concurrent
+calls on one layout (more in flight than the layout's work counters), invalid
+arguments that launch nothing, and the bounded-wait time-out path.
+Tolerances: max |d| <= 1e-2 and mean |d| <= 1e-3 on o and lse; layouts
+bit-exact (checked on the CPU side).
 """
 import math
 
