@@ -34,7 +34,7 @@ STATUS_NAMES = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_SHAPE", 3: "B
                 4: "BSA_ERR_NONCAUSAL", 5: "BSA_ERR_CUDA", 6: "BSA_ERR_OOM",
                 7: "BSA_ERR_DEVICE_TIMEOUT"}
 
-EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_csc", "bsa_layout_order",
+EXPORTED = ["bsa_build_layout", "bsa_layout_csr", "bsa_layout_csc", "bsa_layout_order", "bsa_layout_work",
             "bsa_layout_segments", "bsa_forward", "bsa_forward_host", "bsa_forward_noalloc", "bsa_backward",
             "bsa_decode",
             "bsa_bsbr_workspace_bytes", "bsa_bsbr_retrieval", "bsa_get_status", "bsa_debug_timeout_probe",
@@ -82,6 +82,9 @@ def load_library(path: str = LIB_PATH):
         lib.bsa_layout_order.argtypes = [P, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
                                          ctypes.POINTER(I)]
         lib.bsa_layout_order.restype = I
+        lib.bsa_layout_work.argtypes = [P, ctypes.POINTER(ctypes.POINTER(ctypes.c_int32)),
+                                        ctypes.POINTER(I)]
+        lib.bsa_layout_work.restype = I
         lib.bsa_forward.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P]
         lib.bsa_forward.restype = I
         lib.bsa_forward_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, F, P, P, P]
@@ -208,6 +211,15 @@ def bsa_layout_order(layout: int) -> np.ndarray:
     cnt = ctypes.c_int()
     _check(lib.bsa_layout_order(layout, ctypes.byref(od), ctypes.byref(cnt)))
     return np.ctypeslib.as_array(od, shape=(cnt.value,)).copy()
+
+
+def bsa_layout_work(layout: int) -> np.ndarray:
+    """The forward's work table as an int32 array [layout_heads * nb, 4]."""
+    lib = load_library()
+    wk = ctypes.POINTER(ctypes.c_int32)()
+    cnt = ctypes.c_int()
+    _check(lib.bsa_layout_work(layout, ctypes.byref(wk), ctypes.byref(cnt)))
+    return np.ctypeslib.as_array(wk, shape=(cnt.value * 4,)).copy().reshape(cnt.value, 4)
 
 
 def bsa_forward(q, k, v, layout: int, B: int, n: int, heads: int, kv_heads: int, d: int,

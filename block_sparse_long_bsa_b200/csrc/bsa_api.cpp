@@ -165,6 +165,13 @@ int bsa_layout_order(const bsa_layout* layout, const int32_t** order, int* count
   return BSA_OK;
 }
 
+int bsa_layout_work(const bsa_layout* layout, const int32_t** work, int* count) {
+  if (!layout) return set_error(BSA_ERR_INVALID_ARG, "layout is NULL");
+  if (work) *work = layout->work.data();
+  if (count) *count = int(layout->work.size() / 4);
+  return BSA_OK;
+}
+
 int bsa_layout_csc(const bsa_layout* layout, const int32_t** col_ptr, const int32_t** row_idx,
                    int* cols, int* nnz) {
   if (!layout) return set_error(BSA_ERR_INVALID_ARG, "layout is NULL");

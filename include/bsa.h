@@ -118,6 +118,14 @@ int bsa_layout_csr(const bsa_layout* layout, const int32_t** row_ptr,
  * query block processed at rank r for layout head h.  count = layout_heads*nb. */
 int bsa_layout_order(const bsa_layout* layout, const int32_t** order, int* count);
 
+/* Read-only host view of the forward's work table: for layout head h and rank
+ * r in the longest-row-first order, work[4*(h*nb + r) .. +3] = (query block
+ * order[h*nb + r], its first entry in col_idx, its kept-block count, 1 if its
+ * last kept block is the diagonal one else 0): one work item of bsa_forward
+ * decodes from one such entry.  count = layout_heads*nb entries (4 words
+ * each); uploaded with the layout and staged by bsa_forward_noalloc. */
+int bsa_layout_work(const bsa_layout* layout, const int32_t** work, int* count);
+
 /* Read-only host view of the transposed layout: for layout head h and key
  * block j, row_idx[col_ptr[h*nb + j] .. col_ptr[h*nb + j + 1]) lists, in
  * ascending order, the query blocks whose rows keep j (the key/value side of

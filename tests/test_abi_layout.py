@@ -281,3 +281,31 @@ def test_random_specs_bit_exact_sweep(lib):
         want_ptr, want = _segments_from_csc(ocp, L, nb)
         np.testing.assert_array_equal(seg_ptr, want_ptr, err_msg=label)
         np.testing.assert_array_equal(segs.reshape(-1, 3), want, err_msg=label)
+
+@pytest.mark.parametrize("kind,n,B,L,kw", [
+    (OL.DYADIC, 32768, 64, 1, dict(window=2, global_first=1, dyadic_kmin=2)),
+    (OL.BAND_GLOBAL, 32768, 128, 1, dict(window=2, global_first=1)),
+    (OL.RANDOM, 128 * 300, 128, 3, dict(density=0.3, seed=7)),
+    (OL.BAND_GLOBAL, 1000, 64, 2, dict(window=0, global_first=0)),
+    (OL.BAND_GLOBAL, 1, 64, 1, dict(window=3, global_first=1)),
+    (OL.RANDOM, 64 * 50, 64, 2, dict(density=0.0, seed=1)),
+])
+def test_work_table_decodes_the_oracle_layout(lib, kind, n, B, L, kw):
+    """Each entry of the forward's work table is (query block at that rank of
+    the longest-first order, its first CSR entry, its kept-block count, whether
+    its last kept block is the diagonal), read off the oracle's CSR; the
+    longest-first order is checked on its own above."""
+    lay = bsa.Layout(kind, n, B, L, -1, **kw)
+    work = bsa.bsa_layout_work(lay.handle)
+    order = lay.order()
+    lay.close()
+    nb = OL.n_blocks(n, B)
+    rp, ci = OL.to_csr(OL.kept_sets(kind, n, B, L, **kw))
+    assert work.shape == (L * nb, 4)
+    for h in range(L):
+        for rank in range(nb):
+            row = int(order[h * nb + rank])
+            r = h * nb + row
+            start, length = rp[r], rp[r + 1] - rp[r]
+            diag = int(length > 0 and ci[start + length - 1] == row)
+            assert work[h * nb + rank].tolist() == [row, start, length, diag], (h, rank)
